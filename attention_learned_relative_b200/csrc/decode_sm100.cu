@@ -1,0 +1,387 @@
+// decode_sm100.cu -- single-query decode against a long bf16 KV cache: split-KV
+// streaming kernel plus a log-sum-exp combine kernel.
+//
+// One new query per sequence sits at position n_ctx-1; its own key and value are
+// the cache's last row (the 1,048,576-token context of the archdiff.com model
+// card).  Logit of cache row j: scale * q.k_j + (n_ctx-1-j < R ? r * w[h, n_ctx-1-j]
+// : 0) -- the bias exists only for the last R rows, content-only beyond
+// ("Learned Relative-Position Bias", codewithdark, "Hybrid Attention Interaction").
+//
+// Work: grid (split, key/value head g, sequence b).  A CTA streams a contiguous
+// range of 32-key chunks of K and V once, through a 12-stage TMA ring, and serves
+// all query heads of the group from each chunk (grouped-query attention).  Keys
+// sit on the M dimension of m16n8k16 tensor-core MMAs and the (up to 8) query
+// heads of the group on N:  S^T = K q^T,  O^T += V^T P^T.  P^T's accumulator
+// fragments become B operands through a movmatrix transpose.  The four consumer
+// warps take chunks round-robin and merge their running (max, sum, output) in
+// shared memory; each CTA writes one partial per query head to the workspace.  The
+// combine kernel merges the partials of a (b, h) with one warp.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace relbias {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kChunk = 32;                 // keys per stage
+constexpr int kConsumers = 4;
+// Chunk li lives in stage li % kDStages and is consumed by warp li % kConsumers.
+// kDStages is a multiple of kConsumers, so every stage is always consumed by the
+// same warp, in order: no consumer can look at a stage's barrier while it is two
+// phases behind (which a parity wait could not tell apart from "ready").
+constexpr int kDStages = 12;
+static_assert(kDStages % kConsumers == 0, "stage ownership must be per warp");
+constexpr int kDThreads = (kConsumers + 1) * 32;
+constexpr int kBoxBytes = kChunk * 128;    // 32 keys x 64 bf16
+constexpr int kStageBytes = 4 * kBoxBytes; // K (2 boxes) + V (2 boxes)
+constexpr int kMT = kChunk / 16;           // 16-key MMA tiles per chunk
+constexpr int kRec = kD + 4;               // workspace record: O[128], m, l, pad
+
+struct DecodeBars {
+    uint64_t full[kDStages];
+    uint64_t empty[kDStages];
+    int abort_flag;
+};
+
+struct DecodeSmem {
+    uint8_t stages[kDStages][kStageBytes];
+    float warp_o[kConsumers][8][kD];
+    float warp_m[kConsumers][8];
+    float warp_l[kConsumers][8];
+    DecodeBars bars;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Byte offset of 16-byte chunk (key row, head-dim column dcol) inside a stage half
+// (K or V) loaded as two 64-column boxes with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz(int key, int dcol) {
+    const int box = dcol >> 6;
+    const int ch = (dcol & 63) >> 3;
+    return box * kBoxBytes + key * 128 + ((ch ^ (key & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kDThreads, 1)
+    decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const DecodeParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    DecodeSmem* sm =
+        reinterpret_cast<DecodeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DecodeBars* bars = &sm->bars;
+    volatile int* abort_flag = &bars->abort_flag;
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(p.nchunks, c_begin + p.chunks_per_split);
+    const int nloc = c_end - c_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumers) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            for (int li = 0; li < nloc; ++li) {
+                const int st = li % kDStages;
+                const uint32_t ph = (li / kDStages) & 1;
+                if (!mbar_wait(&bars->empty[st], ph ^ 1, abort_flag)) break;
+                const int key0 = p.key_lo + (c_begin + li) * kChunk;
+                mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
+                uint8_t* base = sm->stages[st];
+                tma_load_4d(base, &tm_k, &bars->full[st], 0, g, key0, b);
+                tma_load_4d(base + kBoxBytes, &tm_k, &bars->full[st], 64, g, key0, b);
+                tma_load_4d(base + 2 * kBoxBytes, &tm_v, &bars->full[st], 0, g, key0, b);
+                tma_load_4d(base + 3 * kBoxBytes, &tm_v, &bars->full[st], 64, g, key0, b);
+            }
+            // Do not leave while copies into this CTA's shared memory are in flight.
+            int dummy = 0;
+            for (int li = max(0, nloc - kDStages); li < nloc; ++li)
+                mbar_wait(&bars->full[li % kDStages], (li / kDStages) & 1, &dummy);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int gq = lane >> 2;        // fragment row group
+    const int qq = lane & 3;         // fragment column pair
+    const float c1 = p.scale_log2;
+
+    // q^T as B fragments (head dim = K, heads of the group = N), padded with zero heads.
+    uint32_t qb[kD / 16][2];
+    {
+        const int n = gq;
+        const bool valid = n < p.G;
+        const __nv_bfloat16* qrow = p.q + (static_cast<size_t>(b) * p.Hq + g * p.G + (valid ? n : 0)) * kD;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            uint32_t lo = valid ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * qq) : 0u;
+            uint32_t hi = valid ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * qq) : 0u;
+            qb[ks][0] = lo;
+            qb[ks][1] = hi;
+        }
+    }
+    // Bias feature of the two heads this thread's accumulator columns belong to.
+    float rs[2];
+    int hcol[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int n = 2 * qq + e;
+        hcol[e] = g * p.G + min(n, p.G - 1);
+        rs[e] = (n < p.G) ? __ldg(p.r + static_cast<size_t>(b) * p.Hq + g * p.G + n) * p.inv_scale : 0.0f;
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.0f, 0.0f};
+    float oacc[kD / 16][4];
+#pragma unroll
+    for (int dt = 0; dt < kD / 16; ++dt) oacc[dt][0] = oacc[dt][1] = oacc[dt][2] = oacc[dt][3] = 0.0f;
+
+    const int last = p.N - 1;
+    bool ok = true;
+    for (int li = warp; li < nloc; li += kConsumers) {
+        const int st = li % kDStages;
+        const uint32_t ph = (li / kDStages) & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->full[st], ph, abort_flag));
+        if (!ok) break;
+        const uint32_t kbase = smem_u32(sm->stages[st]);
+        const uint32_t vbase = kbase + 2 * kBoxBytes;
+        const int key0 = p.key_lo + (c_begin + li) * kChunk;
+
+        // S^T = K q^T for the chunk's groups of 16 keys.
+        float sacc[kMT][4];
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+            sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.0f;
+            const int mi = lane >> 3;
+            const int key = mt * 16 + (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                uint32_t a[4];
+                ldsm_x4(kbase + swz(key, ks * 16 + ((mi >> 1) << 3)), a);
+                mma_bf16(sacc[mt], a, qb[ks][0], qb[ks][1]);
+            }
+        }
+
+        // Logits in log2 units, bias on the last R rows, mask rows past the cache end.
+        const bool biased = key0 + kChunk - 1 >= p.N - p.R;
+        float mc[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = key0 + mt * 16 + gq + ((e >> 1) << 3);
+                const int col = e & 1;
+                float x = sacc[mt][e];
+                if (biased) {
+                    const int dist = last - key;
+                    if (dist >= 0 && dist < p.R)
+                        x = fmaf(rs[col], __ldg(p.w + static_cast<size_t>(hcol[col]) * p.R + dist), x);
+                }
+                x = (key <= last) ? x * c1 : -INFINITY;
+                sacc[mt][e] = x;
+                mc[col] = fmaxf(mc[col], x);
+            }
+        }
+#pragma unroll
+        for (int col = 0; col < 2; ++col) {
+            mc[col] = fmaxf(mc[col], __shfl_xor_sync(0xffffffffu, mc[col], 4));
+            mc[col] = fmaxf(mc[col], __shfl_xor_sync(0xffffffffu, mc[col], 8));
+            mc[col] = fmaxf(mc[col], __shfl_xor_sync(0xffffffffu, mc[col], 16));
+        }
+        float base[2];
+#pragma unroll
+        for (int col = 0; col < 2; ++col) {
+            const float m_new = fmaxf(m_run[col], mc[col]);
+            const float alpha = (m_new == -INFINITY) ? 1.0f : ex2_approx(m_run[col] - m_new);
+            l_run[col] *= alpha;
+#pragma unroll
+            for (int dt = 0; dt < kD / 16; ++dt) {
+                oacc[dt][col] *= alpha;
+                oacc[dt][col + 2] *= alpha;
+            }
+            m_run[col] = m_new;
+            base[col] = (m_new == -INFINITY) ? 0.0f : m_new;
+        }
+        // P^T (keys x heads) -> bf16 -> transposed 8x8 blocks = B fragments.
+        uint32_t pb[kMT][2];
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+            const float p0 = ex2_approx(sacc[mt][0] - base[0]);
+            const float p1 = ex2_approx(sacc[mt][1] - base[1]);
+            const float p2 = ex2_approx(sacc[mt][2] - base[0]);
+            const float p3 = ex2_approx(sacc[mt][3] - base[1]);
+            l_run[0] += p0 + p2;
+            l_run[1] += p1 + p3;
+            pb[mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+            pb[mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+        }
+        // O^T += V^T P^T, head dim in 8 tiles of 16.
+#pragma unroll
+        for (int dt = 0; dt < kD / 16; ++dt) {
+            const int mi = lane >> 3;
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+                const int key = mt * 16 + (lane & 7) + ((mi >> 1) << 3);
+                uint32_t a[4];
+                ldsm_x4_trans(vbase + swz(key, dt * 16 + ((mi & 1) << 3)), a);
+                mma_bf16(oacc[dt], a, pb[mt][0], pb[mt][1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[st]);
+    }
+
+    // Per-warp partial -> shared memory.
+#pragma unroll
+    for (int col = 0; col < 2; ++col) {
+        float lsum = l_run[col];
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+        const int n = 2 * qq + col;
+        if (gq == 0) {
+            sm->warp_m[warp][n] = m_run[col];
+            sm->warp_l[warp][n] = lsum;
+        }
+#pragma unroll
+        for (int dt = 0; dt < kD / 16; ++dt) {
+            sm->warp_o[warp][n][dt * 16 + gq] = oacc[dt][col];
+            sm->warp_o[warp][n][dt * 16 + gq + 8] = oacc[dt][col + 2];
+        }
+    }
+    named_bar_sync(1, kConsumers * 32);
+
+    // Merge the four warps; one partial per (b, head) of the group.
+    const int tid = threadIdx.x;            // 0..127
+    const int n = tid >> 4;                 // head within group (8 x 16 threads)
+    const int d0 = (tid & 15) * 8;
+    if (n < p.G && ok) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sm->warp_m[w][n]);
+        float sc[kConsumers];
+        float Lsum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) {
+            sc[w] = (sm->warp_m[w][n] == -INFINITY) ? 0.0f : ex2_approx(sm->warp_m[w][n] - M);
+            Lsum += sm->warp_l[w][n] * sc[w];
+        }
+        const int h = g * p.G + n;
+        float* rec = p.part + ((static_cast<size_t>(b) * p.Hq + h) * p.nsplit + split) * kRec;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w) acc = fmaf(sm->warp_o[w][n][d0 + e], sc[w], acc);
+            rec[d0 + e] = acc;
+        }
+        if ((tid & 15) == 0) {
+            rec[kD] = M;
+            rec[kD + 1] = Lsum;
+        }
+    }
+}
+
+// One warp per (b, h): merge nsplit partials by log-sum-exp.
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+    const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (wid >= p.B * p.Hq) return;
+    const float* recs = p.part + static_cast<size_t>(wid) * p.nsplit * kRec;
+    float M = -INFINITY;
+    for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, recs[s * kRec + kD]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.0f;
+    for (int s = lane; s < p.nsplit; s += 32) {
+        const float ms = recs[s * kRec + kD];
+        if (ms != -INFINITY) L += recs[s * kRec + kD + 1] * ex2_approx(ms - M);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < p.nsplit; ++s) {
+        const float ms = recs[s * kRec + kD];
+        const float sc = (ms == -INFINITY) ? 0.0f : ex2_approx(ms - M);
+        const float4 o4 = *reinterpret_cast<const float4*>(recs + s * kRec + lane * 4);
+        acc.x = fmaf(o4.x, sc, acc.x);
+        acc.y = fmaf(o4.y, sc, acc.y);
+        acc.z = fmaf(o4.z, sc, acc.z);
+        acc.w = fmaf(o4.w, sc, acc.w);
+    }
+    const float inv = 1.0f / L;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 out;
+    out.x = *reinterpret_cast<uint32_t*>(&lo);
+    out.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p.o + static_cast<size_t>(wid) * kD + lane * 4) = out;
+    if (p.lse != nullptr && lane == 0) p.lse[wid] = (M + __log2f(L)) * kLn2;
+}
+
+}  // namespace
+
+int decode_num_splits(int B, int Hkv, int N, int window, int num_sms) {
+    const int key_lo = window > 0 ? max(0, N - window) : 0;
+    const int nchunks = (N - key_lo + kChunk - 1) / kChunk;
+    const int target = num_sms * 8;   // eight full waves at one CTA per SM
+    const int pairs = B * Hkv;
+    int nsplit = (target + pairs - 1) / pairs;
+    nsplit = max(1, min(nsplit, nchunks));
+    const int cps = (nchunks + nsplit - 1) / nsplit;
+    return (nchunks + cps - 1) / cps;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int nsplit, int d) {
+    return static_cast<size_t>(B) * Hq * nsplit * (d + 4) * sizeof(float);
+}
+
+cudaError_t launch_decode_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                               cudaStream_t stream) {
+    const int smem = static_cast<int>(sizeof(DecodeSmem)) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nsplit, p.Hkv, p.B);
+    decode_splitkv_kernel<<<grid, kDThreads, smem, stream>>>(tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_combine_kernel<<<(p.B * p.Hq + 3) / 4, 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace relbias

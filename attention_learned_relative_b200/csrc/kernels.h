@@ -1,0 +1,57 @@
+// kernels.h -- internal interface between the C-ABI host layer (relbias_attn.cu)
+// and the kernels.  Not part of the public ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace relbias {
+
+// bf16 tcgen05 prefill (prefill_sm100.cu).
+struct PrefillParams {
+    const float* r;          // [B, T, Hq]
+    const float* w;          // [Hq, R]
+    __nv_bfloat16* o;        // [B, T, Hq, d]
+    float* lse;              // [B, Hq, T] or nullptr
+    int B, T, Hq, Hkv;
+    int G;                   // Hq / Hkv
+    int nslots;              // query heads per work item (2 when G is even, else 1)
+    int HP;                  // G / nslots: head pairs per key/value head
+    int window, R;
+    int n_qt;                // ceil(T / 128)
+    int total_items;         // n_qt * B * Hkv * HP
+    float scale_log2;        // scale * log2(e)
+    float inv_scale;         // 1 / scale
+};
+int prefill_bf16_smem_bytes(int d, int R);
+cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                      const PrefillParams& p, int d, int grid, cudaStream_t stream);
+
+// fp32 SIMT prefill (prefill_fp32.cu).
+cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
+                                float* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
+                                float scale, cudaStream_t stream);
+
+// bf16 split-KV decode + log-sum-exp combine (decode_sm100.cu).
+struct DecodeParams {
+    const __nv_bfloat16* q;  // [B, Hq, d]
+    const float* r;          // [B, Hq]
+    const float* w;          // [Hq, R]
+    __nv_bfloat16* o;        // [B, Hq, d]
+    float* lse;              // [B, Hq] or nullptr
+    float* part;             // [B, Hq, nsplit, d + 4] workspace records
+    int B, N, Hq, Hkv, G;
+    int window, R;
+    int key_lo;              // first attended cache row
+    int nchunks;             // kChunk-key chunks in [key_lo, N)
+    int nsplit;              // CTAs per (b, key/value head)
+    int chunks_per_split;
+    float scale_log2;
+    float inv_scale;
+};
+int decode_num_splits(int B, int Hkv, int N, int window, int num_sms);
+size_t decode_workspace_bytes(int B, int Hq, int nsplit, int d);
+cudaError_t launch_decode_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                               cudaStream_t stream);
+
+}  // namespace relbias

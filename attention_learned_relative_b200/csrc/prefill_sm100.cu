@@ -1,0 +1,424 @@
+// prefill_sm100.cu -- bf16 prefill kernel for sm_100a: TMA-staged Q/K/V tiles,
+// tcgen05 MMAs with accumulators in tensor memory, the relative-position bias
+// added to the logits in registers, online softmax, causal / sliding-window tile
+// skipping, and bias evaluation only on tiles that reach distances below R.
+//
+// The bias is produced "inside the tiled loop, block by block, as the scores
+// form", as the essay "Thinking Machines dropped RoPE" says a fused kernel must
+// (its closing section on kernel cost); logits are scale*q.k + r_i*w[h, i-j] for
+// 0 <= i-j < R and scale*q.k beyond (recipe steps 3-5).
+//
+// Work item: (sequence b, key/value head g, a pair of query heads of that group,
+// a 128-row query tile).  The two heads ("slots") share every K/V tile.
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue of slot 0 (TMEM lanes 0-127, one row per thread)
+//   warps 4-7  softmax + epilogue of slot 1
+//   warp 8     TMA producer (Q per item, K and V per tile, 2-stage ring each)
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D);
+// the softmax writes P (bf16, packed in pairs) over the first 64 columns of its S.
+// MMA issue order per KV tile j:  QK0(j)  PV1(j-1)  QK1(j)  PV0(j), so one slot's
+// softmax overlaps the other slot's MMAs.  tcgen05.mma ops from one thread run in
+// issue order, so QK_s(j+1) may overwrite P_s(j) once PV_s(j) has been issued, and
+// when S_s(j) is complete, O_s holds everything up to PV_s(j-1) (softmax may
+// rescale it before releasing P_s(j)).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace relbias {
+
+namespace {
+
+constexpr int kBM = 128;            // query rows per tile (= TMEM lanes)
+constexpr int kBN = 128;            // keys per tile
+constexpr int kStages = 2;          // K and V ring depth
+constexpr int kThreads = 320;
+constexpr int kPadL = 128;          // distance dd lives at table[dd + kPadL]
+constexpr int kTabExtra = 384;      // zeros around the R entries (covers -127 .. R+254)
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows by > 2^8
+
+__host__ __device__ constexpr int tab_floats(int R) { return ((R + kTabExtra + 31) / 32) * 32; }
+
+template <int D>
+struct Layout {
+    static constexpr int kTile = kBM * D * 2;     // bytes of one 128 x D bf16 tile
+    static constexpr int kBox = kBM * 128;        // bytes of one 128-row x 64-col TMA box
+    static constexpr int kQ = 0;                  // 2 slots
+    static constexpr int kK = kQ + 2 * kTile;     // kStages
+    static constexpr int kV = kK + kStages * kTile;
+    static constexpr int kTab = kV + kStages * kTile;
+};
+
+struct Bars {
+    uint64_t q_full, q_empty;
+    uint64_t k_full[kStages], k_empty[kStages];
+    uint64_t v_full[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_full[2], o_final[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Item {
+    int qt, b, g, hp;
+};
+
+__device__ __forceinline__ Item decode_item(const PrefillParams& p, int u) {
+    const int per_qt = p.B * p.Hkv * p.HP;
+    const int qr = u / per_qt;
+    int rem = u - qr * per_qt;
+    Item it;
+    it.qt = p.n_qt - 1 - qr;   // heaviest query tiles first
+    it.b = rem / (p.Hkv * p.HP);
+    rem -= it.b * p.Hkv * p.HP;
+    it.g = rem / p.HP;
+    it.hp = rem - it.g * p.HP;
+    return it;
+}
+
+// First key tile and number of key tiles a query tile visits.
+__device__ __forceinline__ void kv_range(const PrefillParams& p, int i0, int& j_first, int& ntiles) {
+    int lo = 0;
+    if (p.window > 0) lo = max(0, i0 - p.window + 1);
+    j_first = (lo / kBN) * kBN;
+    ntiles = (i0 - j_first) / kBN + 1;
+}
+
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * Layout<D>::kBox;
+        const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
+        const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
+        umma_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, uint32_t idesc,
+                                         bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < kBN / 16; ++kk) {
+        // V tile: keys are the K dimension (8-row groups 1024 B apart), head dim
+        // is the N dimension (64-column TMA boxes kBox apart): MN-major operand.
+        const uint64_t b = smem_desc_sw128(v_addr + kk * 16 * 128, Layout<D>::kBox, 1024);
+        umma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+    using L = Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tabn = tab_floats(p.R);
+    float* tables = reinterpret_cast<float*>(smem + L::kTab);
+    Bars* bars = reinterpret_cast<Bars*>(smem + L::kTab + 2 * tabn * 4);
+    volatile int* abort_flag = &bars->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->s_full[s], 1);
+            mbar_init(&bars->p_full[s], kBM);
+            mbar_init(&bars->o_final[s], 1);
+        }
+        mbar_init(&bars->mma_done, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_base;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int kv_it = 0, item_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
+                const Item it = decode_item(p, u);
+                const int i0 = it.qt * kBM;
+                int j_first, ntiles;
+                kv_range(p, i0, j_first, ntiles);
+                const int h0 = it.g * p.G + it.hp * p.nslots;
+                if (item_it > 0 && !(ok = mbar_wait(&bars->q_empty, (item_it - 1) & 1, abort_flag))) break;
+                mbar_arrive_expect_tx(&bars->q_full, p.nslots * L::kTile);
+                for (int s = 0; s < p.nslots; ++s)
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full, bx * 64,
+                                    h0 + s, i0, it.b);
+                for (int t = 0; t < ntiles; ++t, ++kv_it) {
+                    const int st = kv_it & 1;
+                    const uint32_t ph = (kv_it >> 1) & 1;
+                    const int j0 = j_first + t * kBN;
+                    if (!(ok = mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag))) break;
+                    mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st], bx * 64,
+                                    it.g, j0, it.b);
+                    if (!(ok = mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag))) break;
+                    mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st], bx * 64,
+                                    it.g, j0, it.b);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+            const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
+            const uint32_t s_tm[2] = {tmem_base, tmem_base + 128};
+            const uint32_t o_tm[2] = {tmem_base + 256, tmem_base + 384};
+            const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
+            int kv_it = 0, item_it = 0;
+            uint32_t pcnt[2] = {0, 0};
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
+                const Item it = decode_item(p, u);
+                int j_first, ntiles;
+                kv_range(p, it.qt * kBM, j_first, ntiles);
+                if (!(ok = mbar_wait(&bars->q_full, item_it & 1, abort_flag))) break;
+                tc_fence_after();
+                int prev_st = 0;
+                for (int t = 0; t < ntiles; ++t, ++kv_it) {
+                    const int st = kv_it & 1;
+                    const uint32_t ph = (kv_it >> 1) & 1;
+                    const uint32_t k_addr = smem_u32(smem + L::kK + st * L::kTile);
+                    const uint32_t v_addr = smem_u32(smem + L::kV + st * L::kTile);
+                    if (!(ok = mbar_wait(&bars->k_full[st], ph, abort_flag))) break;
+                    tc_fence_after();
+                    issue_qk<D>(s_tm[0], q_addr[0], k_addr, idesc_qk);
+                    umma_commit(&bars->s_full[0]);
+                    if (p.nslots == 2) {
+                        if (t > 0) {
+                            if (!(ok = mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag))) break;
+                            ++pcnt[1];
+                            tc_fence_after();
+                            issue_pv<D>(o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv,
+                                        t - 1 > 0);
+                            umma_commit(&bars->v_empty[prev_st]);
+                        }
+                        issue_qk<D>(s_tm[1], q_addr[1], k_addr, idesc_qk);
+                        umma_commit(&bars->s_full[1]);
+                    }
+                    umma_commit(&bars->k_empty[st]);
+                    if (t == ntiles - 1) umma_commit(&bars->q_empty);
+                    if (!(ok = mbar_wait(&bars->v_full[st], ph, abort_flag))) break;
+                    if (!(ok = mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag))) break;
+                    ++pcnt[0];
+                    tc_fence_after();
+                    issue_pv<D>(o_tm[0], s_tm[0], v_addr, idesc_pv, t > 0);
+                    if (p.nslots == 1) umma_commit(&bars->v_empty[st]);
+                    if (t == ntiles - 1) umma_commit(&bars->o_final[0]);
+                    prev_st = st;
+                }
+                if (ok && p.nslots == 2) {
+                    if (!(ok = mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag))) break;
+                    ++pcnt[1];
+                    tc_fence_after();
+                    issue_pv<D>(o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv, ntiles > 1);
+                    umma_commit(&bars->v_empty[prev_st]);
+                    umma_commit(&bars->o_final[1]);
+                }
+            }
+            // Drain: wait (bounded, regardless of abort) until every MMA issued has finished.
+            umma_commit(&bars->mma_done);
+            int dummy = 0;
+            mbar_wait(&bars->mma_done, 0, &dummy);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax / epilogue
+        const int slot = threadIdx.x >> 7;
+        const int t = threadIdx.x & 127;
+        const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
+        const uint32_t s_tm = tmem_base + lane_off + slot * 128;
+        const uint32_t o_tm = tmem_base + lane_off + 256 + slot * 128;
+        float* wtab = tables + slot * tabn;
+        const float c1 = p.scale_log2;
+        int tile_it = 0, item_it = 0;
+        bool ok = slot < p.nslots;
+        for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
+            const Item it = decode_item(p, u);
+            const int i0 = it.qt * kBM;
+            int j_first, ntiles;
+            kv_range(p, i0, j_first, ntiles);
+            const int h = it.g * p.G + it.hp * p.nslots + slot;
+
+            // This head's distance table, zero outside [0, R), staged once per item.
+            named_bar_sync(1 + slot, kBM);
+            for (int x = t; x < tabn; x += kBM) {
+                const int dd = x - kPadL;
+                wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(p.w + static_cast<size_t>(h) * p.R + dd) : 0.0f;
+            }
+            named_bar_sync(1 + slot, kBM);
+
+            const int i = i0 + t;
+            const bool row_ok = i < p.T;
+            const float rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale
+                                    : 0.0f;
+            float m_used = -INFINITY;   // running max, log2 units
+            float l = 0.0f;
+
+            for (int tt = 0; tt < ntiles; ++tt, ++tile_it) {
+                const int j0 = j_first + tt * kBN;
+                const int delta0 = i0 - j0;   // distance of (row t, key c) is delta0 + t - c
+                ok = warp_all(mbar_wait(&bars->s_full[slot], tile_it & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sr[kBN];
+#pragma unroll
+                for (int c = 0; c < kBN; c += 32) tmem_ld32(s_tm + c, sr + c);
+                tmem_ld_wait();
+                float s[kBN];
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+
+                if (delta0 - (kBN - 1) < p.R) {
+                    // Some key of this tile is closer than R: add r_i * w[h, i-j] (in units
+                    // of the unscaled logit; the table is zero outside [0, R)).
+                    const float* wp = wtab + kPadL + delta0 + t;
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c) s[c] = fmaf(rs, wp[-c], s[c]);
+                }
+                if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
+                    const int hi = delta0 + t;   // causal: key c visible iff c <= hi
+                    const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
+                }
+                float mx = s[0];
+#pragma unroll
+                for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+                const float m_tile = mx * c1;
+                const bool grow = m_tile > m_used + kRescaleThreshold;
+                float alpha = 1.0f;
+                if (grow) {
+                    alpha = ex2_approx(m_used - m_tile);
+                    l *= alpha;
+                    m_used = m_tile;
+                }
+                if (tt > 0 && __any_sync(0xffffffffu, grow)) {
+                    // O holds every PV up to the previous tile: rescale it in place.
+                    uint32_t ob[32];
+#pragma unroll
+                    for (int c = 0; c < D; c += 32) {
+                        tmem_ld32(o_tm + c, ob);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+                        tmem_st32(o_tm + c, ob);
+                    }
+                    tmem_st_wait();
+                }
+                const float mb = (m_used == -INFINITY) ? 0.0f : m_used;
+                uint32_t pk[kBN / 2];
+#pragma unroll
+                for (int c = 0; c < kBN; c += 2) {
+                    const float p0 = ex2_approx(fmaf(s[c], c1, -mb));
+                    const float p1 = ex2_approx(fmaf(s[c + 1], c1, -mb));
+                    l += p0 + p1;
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(s_tm, pk);
+                tmem_st32(s_tm + 32, pk + 32);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[slot]);
+            }
+            if (!ok) break;
+
+            // Epilogue: O / l to bf16, and the row's log-sum-exp.
+            ok = warp_all(mbar_wait(&bars->o_final[slot], item_it & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+            __nv_bfloat16* orow = p.o + ((static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+                uint32_t ob[32];
+                tmem_ld32(o_tm + c, ob);
+                tmem_ld_wait();
+                uint32_t packed[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    packed[e] = pack_bf16x2(__uint_as_float(ob[2 * e]) * inv_l, __uint_as_float(ob[2 * e + 1]) * inv_l);
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                }
+            }
+            if (p.lse != nullptr && row_ok)
+                p.lse[(static_cast<size_t>(it.b) * p.Hq + h) * p.T + i] = (m_used + __log2f(l)) * kLn2;
+            tc_fence_before();
+        }
+    }
+
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace
+
+int prefill_bf16_smem_bytes(int d, int R) {
+    const int lay = d == 64 ? Layout<64>::kTab : Layout<128>::kTab;
+    const int need = lay + 2 * tab_floats(R) * 4 + static_cast<int>(sizeof(Bars)) + 1024;
+    // Each CTA allocates all 512 TMEM columns: never let two CTAs share an SM
+    // (228 KB of shared memory per SM, so more than 114 KB each).
+    return need > 120 * 1024 ? need : 120 * 1024;
+}
+
+cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                      const PrefillParams& p, int d, int grid, cudaStream_t stream) {
+    const int smem = prefill_bf16_smem_bytes(d, p.R);
+    cudaError_t e;
+    if (d == 128) {
+        e = cudaFuncSetAttribute(prefill_bf16_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        prefill_bf16_sm100_kernel<128><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    } else {
+        e = cudaFuncSetAttribute(prefill_bf16_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        prefill_bf16_sm100_kernel<64><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace relbias

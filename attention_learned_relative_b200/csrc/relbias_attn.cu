@@ -1,0 +1,258 @@
+// relbias_attn.cu -- the C ABI of librelbias_attn.so (declared in
+// include/relbias_attn.h): argument checks, TMA descriptor set-up, launch
+// configuration and error reporting.  The kernels are compiled into this one
+// translation unit so they share the device-side status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "relbias_attn.h"
+
+#include "decode_sm100.cu"
+#include "prefill_fp32.cu"
+#include "prefill_sm100.cu"
+
+namespace relbias {
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(RELBIAS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(std::string& why) {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    static std::string err;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || ptr == nullptr)
+            err = std::string("cuTensorMapEncodeTiled unavailable: ") + cudaGetErrorString(e);
+        else
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    why = err;
+    return fn;
+}
+
+struct DeviceInfo {
+    int major = 0, minor = 0, sms = 0;
+};
+
+int device_info(DeviceInfo& info) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if ((e = cudaDeviceGetAttribute(&info.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&info.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    return RELBIAS_OK;
+}
+
+// 4-D bf16 tensor map over a [B, T, H, d] tensor, box = 64 head-dim columns x
+// `rows` tokens of one head, 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int d, int rows) {
+    std::string why;
+    EncodeTiledFn fn = encode_fn(why);
+    if (fn == nullptr) return fail(RELBIAS_ERR_CUDA, "%s", why.c_str());
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                             static_cast<cuuint64_t>(T) * H * d * 2};
+    cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(RELBIAS_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return RELBIAS_OK;
+}
+
+int check_common(int B, int T, int Hq, int Hkv, int d, int R, float scale, const float* w) {
+    if (B < 0 || T < 0) return fail(RELBIAS_ERR_ARG, "B (%d) and T (%d) must be >= 0", B, T);
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+        return fail(RELBIAS_ERR_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
+    if (d < 1) return fail(RELBIAS_ERR_ARG, "d (%d) must be positive", d);
+    if (R < 0) return fail(RELBIAS_ERR_ARG, "R (%d) must be >= 0", R);
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(RELBIAS_ERR_ARG, "scale (%g) must be positive and finite", static_cast<double>(scale));
+    if (R > 0 && (w == nullptr || !aligned4(w))) return fail(RELBIAS_ERR_ARG, "w is null or misaligned");
+    return RELBIAS_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+}  // namespace relbias
+
+using namespace relbias;
+
+extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, const float* r, const float* w,
+                                void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
+                                float scale, int dtype, void* stream) {
+    t_err.clear();
+    int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0 || T == 0) return RELBIAS_OK;
+    if (!q || !k || !v || !r || !o) return fail(RELBIAS_ERR_ARG, "q, k, v, r and o must not be null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(RELBIAS_ERR_ARG, "q, k, v and o must be 16-byte aligned");
+    if (!aligned4(r) || (lse && !aligned4(lse))) return fail(RELBIAS_ERR_ARG, "r and lse must be 4-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (dtype == RELBIAS_FP32) {
+        if (d != 32 && d != 64 && d != 128 && d != 256)
+            return fail(RELBIAS_ERR_UNSUPPORTED, "fp32 prefill supports d in {32, 64, 128, 256}, got %d", d);
+        cudaError_t e = launch_prefill_fp32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                            static_cast<const float*>(v), r, w, static_cast<float*>(o), lse, B, T,
+                                            Hq, Hkv, d, window, R, scale, st);
+        return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "fp32 prefill launch");
+    }
+
+    if (d != 64 && d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill supports d in {64, 128}, got %d", d);
+    if (R > 2048) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
+    DeviceInfo dev;
+    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill needs compute capability 10.0 (sm_100a), found %d.%d",
+                    dev.major, dev.minor);
+
+    CUtensorMap tq, tk, tv;
+    if ((rc = make_map(&tq, q, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tk, k, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
+
+    PrefillParams p{};
+    p.r = r;
+    p.w = w;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.nslots = (p.G % 2 == 0) ? 2 : 1;
+    p.HP = p.G / p.nslots;
+    p.window = window > 0 ? window : 0;
+    p.R = R;
+    p.n_qt = (T + 127) / 128;
+    const long long items = static_cast<long long>(p.n_qt) * B * Hkv * p.HP;
+    if (items > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", items);
+    p.total_items = static_cast<int>(items);
+    p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
+    const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
+    cudaError_t e = launch_prefill_bf16_sm100(tq, tk, tv, p, d, grid, st);
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "bf16 prefill launch");
+}
+
+extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d, int window) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || n_ctx < 1 || d < 1) return 0;
+    DeviceInfo dev;
+    if (device_info(dev) != RELBIAS_OK) return 0;
+    const int nsplit = decode_num_splits(B, Hkv, n_ctx, window, dev.sms);
+    return decode_workspace_bytes(B, Hq, nsplit, d);
+}
+
+extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const void* v_cache, const float* r,
+                                   const float* w, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d,
+                                   int window, int R, float scale, int dtype, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+    t_err.clear();
+    int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0) return RELBIAS_OK;
+    if (n_ctx < 1) return fail(RELBIAS_ERR_ARG, "n_ctx (%d) must be >= 1", n_ctx);
+    if (!q || !k_cache || !v_cache || !r || !o || !workspace)
+        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, r, o and workspace must not be null");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace))
+        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, o and workspace must be 16-byte aligned");
+    if (!aligned4(r) || (lse && !aligned4(lse))) return fail(RELBIAS_ERR_ARG, "r and lse must be 4-byte aligned");
+    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports bf16 only");
+    if (d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports d == 128, got %d", d);
+    if (Hq / Hkv > 8) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports up to 8 query heads per key/value head");
+    DeviceInfo dev;
+    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "decode needs compute capability 10.0 (sm_100a), found %d.%d", dev.major,
+                    dev.minor);
+
+    DecodeParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.r = r;
+    p.w = w;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.part = static_cast<float*>(workspace);
+    p.B = B;
+    p.N = n_ctx;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.window = window > 0 ? window : 0;
+    p.R = R;
+    p.key_lo = p.window > 0 ? std::max(0, n_ctx - p.window) : 0;
+    p.nchunks = (n_ctx - p.key_lo + kChunk - 1) / kChunk;
+    p.nsplit = decode_num_splits(B, Hkv, n_ctx, p.window, dev.sms);
+    p.chunks_per_split = (p.nchunks + p.nsplit - 1) / p.nsplit;
+    p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
+    const size_t need = decode_workspace_bytes(B, Hq, p.nsplit, d);
+    if (ws_bytes < need)
+        return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes, need);
+
+    CUtensorMap tk, tv;
+    if ((rc = make_map(&tk, k_cache, B, n_ctx, Hkv, d, kChunk)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v_cache, B, n_ctx, Hkv, d, kChunk)) != RELBIAS_OK) return rc;
+    cudaError_t e = launch_decode_bf16(tk, tv, p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "decode launch");
+}
+
+extern "C" const char* relbias_last_error(void) { return t_err.c_str(); }
+
+extern "C" int relbias_device_status(int reset) {
+    t_err.clear();
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    unsigned int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v))) != cudaSuccess)
+        return cuda_fail(e, "reading the status word");
+    if (reset) {
+        const unsigned int zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero))) != cudaSuccess)
+            return cuda_fail(e, "clearing the status word");
+    }
+    return static_cast<int>(v);
+}
+
+extern "C" int relbias_version(void) { return 100; }

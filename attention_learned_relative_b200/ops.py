@@ -1,0 +1,172 @@
+"""Python binding of librelbias_attn.so (ctypes).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity and their device pointers passed to the C entry points declared in
+include/relbias_attn.h.  Every step of the computation runs in the library's CUDA
+kernels; there is no fallback path.  If the shared library is missing the calls
+raise, they never compute anything on the CPU.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librelbias_attn.so")
+
+RELBIAS_OK = 0
+RELBIAS_ERR_ARG = -1
+RELBIAS_ERR_UNSUPPORTED = -2
+RELBIAS_ERR_CUDA = -3
+RELBIAS_STATUS_TIMEOUT = 1
+RELBIAS_BF16 = 0
+RELBIAS_FP32 = 1
+
+# Every symbol include/relbias_attn.h declares: (name, restype, argtypes).
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "relbias_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
+    "relbias_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ,
+                                 _VP]),
+    "relbias_last_error": (ctypes.c_char_p, []),
+    "relbias_device_status": (_I, [_I]),
+    "relbias_version": (_I, []),
+}
+
+_lib = None
+
+
+class RelbiasError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("relbias error %d: %s" % (code, msg))
+        self.code = code
+
+
+def lib():
+    """The loaded shared library (built in-tree by attention_learned_relative_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("%s is missing: build it with `python -m attention_learned_relative_b200.build`"
+                               % LIB_PATH)
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(rc: int):
+    if rc != RELBIAS_OK:
+        raise RelbiasError(rc, lib().relbias_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return RELBIAS_BF16
+    if t.dtype == torch.float32:
+        return RELBIAS_FP32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def attn_fwd(q, k, v, r, w, window: int, R: int, scale: float | None = None, out=None, lse=None,
+             stream=None):
+    """Prefill.  q [B,T,Hq,d], k/v [B,T,Hkv,d] (bf16 or fp32, CUDA, contiguous),
+    r [B,T,Hq] fp32, w [Hq,R] fp32.  Returns o [B,T,Hq,d] (and fills `lse`
+    [B,Hq,T] fp32 when given).  scale defaults to 1/sqrt(d)."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape[:2] == (B, T) and k.shape[3] == d, "k/v shape %s does not match q %s" % (k.shape, q.shape))
+    _need(q.dtype == k.dtype == v.dtype, "q, k, v must share a dtype")
+    _need(r.shape == (B, T, Hq) and r.dtype == torch.float32, "r must be fp32 [B,T,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    for t in (q, k, v, r, w, out, lse):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out.shape == q.shape and out.dtype == q.dtype, "out must match q")
+    _need(lse is None or (lse.shape == (B, Hq, T) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq,T]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
+                                B, T, Hq, Hkv, d, int(window), int(R), float(scale), _dtype_code(q),
+                                _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, n_ctx: int, d: int, window: int) -> int:
+    """Bytes of device scratch relbias_attn_decode needs for this shape (on the current device)."""
+    return int(lib().relbias_attn_decode_workspace_size(B, Hq, Hkv, n_ctx, d, int(window)))
+
+
+def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | None = None, out=None,
+                lse=None, workspace=None, stream=None):
+    """Decode one query per sequence at position n_ctx-1.  q [B,Hq,d] bf16,
+    k_cache/v_cache [B,n_ctx,Hkv,d] bf16, r [B,Hq] fp32, w [Hq,R] fp32.
+    Returns o [B,Hq,d] bf16 (fills `lse` [B,Hq] when given).  `workspace` is a
+    byte tensor of at least decode_workspace_size(...) bytes; allocated if None."""
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "q [B,Hq,d], cache [B,N,Hkv,d]")
+    B, Hq, d = q.shape
+    _, N, Hkv, _ = k_cache.shape
+    _need(k_cache.shape[0] == B and k_cache.shape[3] == d, "cache shape does not match q")
+    _need(q.dtype == k_cache.dtype == v_cache.dtype, "q and cache must share a dtype")
+    _need(r.shape == (B, Hq) and r.dtype == torch.float32, "r must be fp32 [B,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    for t in (q, k_cache, v_cache, r, w, out, lse, workspace):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(lse is None or (lse.shape == (B, Hq) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq]")
+    need = decode_workspace_size(B, Hq, Hkv, N, d, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
+                                   B, N, Hq, Hkv, d, int(window), int(R), float(scale), _dtype_code(q),
+                                   _ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def device_status(reset: bool = True) -> int:
+    """Synchronise and return the kernels' status bits (RELBIAS_STATUS_*)."""
+    rc = lib().relbias_device_status(1 if reset else 0)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def last_error() -> str:
+    return lib().relbias_last_error().decode()
+
+
+def version() -> int:
+    return int(lib().relbias_version())

@@ -1,0 +1,142 @@
+/*
+ * relbias_attn.h -- C ABI of librelbias_attn.so: causal grouped-query attention
+ * with an additive, input-dependent, learned relative-position bias, forward
+ * pass, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch b, query head h, query position i):
+ *
+ *   logit[j] = scale * <q[b,i,h,:], k[b,j,g,:]> + bias[j]          g = h / (Hq/Hkv)
+ *   bias[j]  = r[b,i,h] * w[h, i-j]   if 0 <= i-j < R,   else 0
+ *   j ranges over A_i = { j : 0 <= i-j  and  (window <= 0 or i-j < window) }
+ *   o[b,i,h,:] = sum_j softmax(logit)[j] * v[b,j,g,:]
+ *   lse[b,h,i] = log sum_j exp(logit[j])
+ *
+ * Sources.  The bias is added to the scaled logits before the softmax, next to
+ * the causal mask, and is exactly zero at distances of R or more ("Thinking
+ * Machines dropped RoPE", wpnews.pro essay: the five-step recipe, steps 3-5,
+ * and the relative_position_bias listing).  The per-token, per-head feature r
+ * comes from a fourth projection and is modulated by distance (banandre.com
+ * Inkling deep dive, "No RoPE? No Problem?"); here it multiplies a learned
+ * per-head distance table w.  Local layers use window = 512 and R = 512; global
+ * layers use the full causal mask with R = 1024 and content-only attention
+ * beyond ("Learned Relative-Position Bias", codewithdark concepts page, "Key
+ * Components" and "Hybrid Attention Interaction").  The scaled-logit form is the
+ * T5-style formula on that page ("Standard Relative Bias (T5-style)"); the scale
+ * is a parameter because the essay's logit-scaling sentence lost its symbols.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     densely packed, and at least 16-byte aligned.  The library allocates no
+ *     device memory and keeps no per-call state.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise.  Arguments are checked on the host before
+ *     any launch; a rejected call launches nothing.
+ *   - Return value: RELBIAS_OK (0) or a negative RELBIAS_ERR_* code.  The calls
+ *     never abort the process.  relbias_last_error() describes the last failure
+ *     on the calling thread.
+ *   - Kernels bound every wait on an asynchronous copy or tensor-core result.  A
+ *     wait that runs out records RELBIAS_STATUS_TIMEOUT in a device-side status
+ *     word, the kernel winds down and returns; relbias_device_status() reads it.
+ */
+#ifndef RELBIAS_ATTN_H
+#define RELBIAS_ATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RELBIAS_API __attribute__((visibility("default")))
+#else
+#define RELBIAS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RELBIAS_OK               0
+#define RELBIAS_ERR_ARG         -1  /* null pointer, bad shape, misalignment, bad scale   */
+#define RELBIAS_ERR_UNSUPPORTED -2  /* valid request this build or device cannot serve    */
+#define RELBIAS_ERR_CUDA        -3  /* a CUDA runtime call or kernel launch failed        */
+
+/* Bits of the device-side status word (relbias_device_status). */
+#define RELBIAS_STATUS_TIMEOUT   1u /* a bounded wait inside a kernel ran out             */
+
+/* Element type of q, k, v and o.  r, w and lse are always fp32. */
+typedef enum {
+    RELBIAS_BF16 = 0,   /* bf16 storage, fp32 accumulation (tensor cores)  */
+    RELBIAS_FP32 = 1    /* fp32 storage and arithmetic (CUDA cores)        */
+} relbias_dtype;
+
+/*
+ * Prefill: every query row of every sequence attends causally to its own
+ * sequence.
+ *
+ *   q    [B, T, Hq,  d]   dtype
+ *   k    [B, T, Hkv, d]   dtype
+ *   v    [B, T, Hkv, d]   dtype
+ *   r    [B, T, Hq]       fp32   per-token, per-head bias feature
+ *   w    [Hq, R]          fp32   per-head distance table (may be NULL if R == 0)
+ *   o    [B, T, Hq,  d]   dtype  output, written for every row
+ *   lse  [B, Hq, T]       fp32   natural-log LSE of each row; may be NULL
+ *
+ *   B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0; window <= 0 means full causal;
+ *   R >= 0 (R == 0: no bias); scale > 0 and finite.
+ *   RELBIAS_BF16 needs a B200-class GPU (compute capability 10.0), d in {64, 128}
+ *   and R <= 2048; RELBIAS_FP32 takes d in {32, 64, 128, 256} on any GPU.
+ *   The output buffers must not overlap the inputs.
+ */
+RELBIAS_API int relbias_attn_fwd(const void* q, const void* k, const void* v,
+                     const float* r, const float* w,
+                     void* o, float* lse,
+                     int B, int T, int Hq, int Hkv, int d,
+                     int window, int R, float scale,
+                     int dtype, void* stream);
+
+/*
+ * Decode: one new query per sequence at position n_ctx-1 against a key/value
+ * cache of n_ctx rows whose last row already holds that query's own key and
+ * value (the 1,048,576-token context of the archdiff.com model card, "Context").
+ * The keys are split over many CTAs; each writes a partial (max, sum, output)
+ * into `workspace`, and a second kernel merges the partials by log-sum-exp.
+ *
+ *   q        [B, Hq, d]          bf16
+ *   k_cache  [B, n_ctx, Hkv, d]  bf16
+ *   v_cache  [B, n_ctx, Hkv, d]  bf16
+ *   r        [B, Hq]             fp32   the new token's bias feature
+ *   w        [Hq, R]             fp32   (may be NULL if R == 0)
+ *   o        [B, Hq, d]          bf16
+ *   lse      [B, Hq]             fp32   may be NULL
+ *   workspace, ws_bytes: caller-owned device scratch of at least
+ *            relbias_attn_decode_workspace_size(...) bytes, 16-byte aligned; its
+ *            contents on entry do not matter and are overwritten.
+ *
+ *   dtype must be RELBIAS_BF16; d == 128; Hq/Hkv <= 8; n_ctx >= 1; other
+ *   argument rules as for relbias_attn_fwd.
+ */
+RELBIAS_API size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d,
+                                          int window);
+
+RELBIAS_API int relbias_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const float* r, const float* w,
+                        void* o, float* lse,
+                        int B, int n_ctx, int Hq, int Hkv, int d,
+                        int window, int R, float scale,
+                        int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* Description of the last failed call on this thread ("" if none).  The string
+ * stays valid until the next library call on the same thread. */
+RELBIAS_API const char* relbias_last_error(void);
+
+/* Synchronises the current device, returns the device-side status bits
+ * accumulated since the last reset (RELBIAS_STATUS_*) and, if reset != 0,
+ * clears them.  Returns a negative RELBIAS_ERR_CUDA on a CUDA failure. */
+RELBIAS_API int relbias_device_status(int reset);
+
+/* Library version as major*10000 + minor*100 + patch. */
+RELBIAS_API int relbias_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RELBIAS_ATTN_H */

@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/relbias_attn.h declares, and rejects bad arguments on the host (no CUDA
+call is made before the checks pass)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_learned_relative_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "relbias_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^RELBIAS_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for want in ["relbias_attn_fwd", "relbias_attn_decode", "relbias_attn_decode_workspace_size",
+                 "relbias_last_error", "relbias_device_status", "relbias_version"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(ops.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+        assert name in ops.SIGNATURES, "binding lacks " + name
+
+
+def test_version(lib):
+    assert ops.version() >= 100
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=1, T=8, Hq=4, Hkv=2, d=128,
+             window=0, R=16, scale=0.125, dtype=ops.RELBIAS_BF16)
+    a.update(kw)
+    return lib.relbias_attn_fwd(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"], a["T"],
+                                a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), ops.RELBIAS_ERR_ARG),
+    (dict(Hkv=0), ops.RELBIAS_ERR_ARG),
+    (dict(B=-1), ops.RELBIAS_ERR_ARG),
+    (dict(R=-1), ops.RELBIAS_ERR_ARG),
+    (dict(scale=0.0), ops.RELBIAS_ERR_ARG),
+    (dict(scale=float("inf")), ops.RELBIAS_ERR_ARG),
+    (dict(scale=float("nan")), ops.RELBIAS_ERR_ARG),
+    (dict(q=None), ops.RELBIAS_ERR_ARG),
+    (dict(w=None), ops.RELBIAS_ERR_ARG),
+    (dict(o=FAKE + 8), ops.RELBIAS_ERR_ARG),
+    (dict(k=FAKE + 2), ops.RELBIAS_ERR_ARG),
+    (dict(r=FAKE + 1), ops.RELBIAS_ERR_ARG),
+    (dict(dtype=7), ops.RELBIAS_ERR_ARG),
+    (dict(d=96), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(R=4096), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(d=48, dtype=ops.RELBIAS_FP32), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_on_host(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_empty_inputs_are_a_no_op(lib):
+    assert _fwd(lib, B=0) == ops.RELBIAS_OK
+    assert _fwd(lib, T=0) == ops.RELBIAS_OK
+    assert _fwd(lib, B=0, q=None, k=None, v=None, o=None, r=None) == ops.RELBIAS_OK
+    assert ops.last_error() == ""
+
+
+def test_r0_needs_no_table(lib):
+    # R == 0 with w == NULL passes the argument checks (it then fails only for the
+    # missing device on a CPU-only host, or runs on a GPU host).
+    rc = _fwd(lib, R=0, w=None, d=96)
+    assert rc == ops.RELBIAS_ERR_UNSUPPORTED
+
+
+def _dec(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=2, N=100, Hq=8, Hkv=1, d=128,
+             window=0, R=16, scale=0.1, dtype=ops.RELBIAS_BF16, ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    return lib.relbias_attn_decode(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"], a["N"],
+                                   a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["dtype"],
+                                   a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=0), ops.RELBIAS_ERR_ARG),
+    (dict(ws=None), ops.RELBIAS_ERR_ARG),
+    (dict(ws=FAKE + 4), ops.RELBIAS_ERR_ARG),
+    (dict(Hq=12, Hkv=8), ops.RELBIAS_ERR_ARG),
+    (dict(scale=-1.0), ops.RELBIAS_ERR_ARG),
+    (dict(dtype=ops.RELBIAS_FP32), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(d=64), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(Hq=16, Hkv=1), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_decode_rejects_on_host(lib, kw, code):
+    assert _dec(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_decode_empty_batch(lib):
+    assert _dec(lib, B=0) == ops.RELBIAS_OK
+
+
+def test_workspace_size_rejects_bad_shapes(lib):
+    assert ops.decode_workspace_size(0, 8, 1, 100, 128, 0) == 0
+    assert ops.decode_workspace_size(1, 8, 3, 100, 128, 0) == 0
