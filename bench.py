@@ -1,0 +1,467 @@
+#!/usr/bin/env python3
+"""Benchmark of the relative-position-bias attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the workload's hot path over one batch of synthetic input:
+for the default workload (local-layer prefill: B=2, T=8192, 32 query / 4 key-value
+heads, d=128, window 512, R=512) that is one relbias_attn_fwd call writing O and
+LSE.  Inputs are resident in HBM when the timed region starts; steps rotate over
+several independently drawn input sets so that no step finds the previous step's
+data in the 126 MB L2.  The timed region is K back-to-back steps bracketed by a
+barrier and a device synchronisation on both sides and timed with CUDA events on
+the launching stream; with N GPUs every rank runs its own copy of the workload
+(independent units, no data-path collective: weak scaling) and the time is the max
+over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle instead (the only other code path for
+this method) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "local_prefill_bf16"
+METRIC = "masked TFLOP/s & frac of bf16 tensor peak (prefill); decode HBM GB/s vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: ~2 s of work)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest() -> str:
+    """sha256 over the CUDA sources: ties an ncu capture to the kernels it measured."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_learned_relative_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    if that summary was taken on the current sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_%s.md" % workload)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_sha256:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != source_digest():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """Polls the SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = [("gpu_idle", 0x1), ("applications_clocks_setting", 0x2), ("sw_power_cap", 0x4),
+               ("hw_slowdown", 0x8), ("sync_boost", 0x10), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80)]
+
+    def __init__(self, torch_device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable: " + getattr(self, "error", "")]}
+        names = [n for n, bit in self.REASONS if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def make_sets(wl, nsets, device):
+    import torch
+    from attention_learned_relative_b200 import workloads
+    from dataclasses import replace
+    sets = []
+    for s in range(nsets):
+        x = workloads.make_inputs(replace(wl, seed=wl.seed + 1000 * s), device=device)
+        if wl.decode:
+            x["o"] = torch.empty_like(x["q"])
+            x["lse"] = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
+        else:
+            x["o"] = torch.empty_like(x["q"])
+            x["lse"] = torch.empty(wl.B, wl.Hq, wl.T, dtype=torch.float32, device=device)
+        sets.append(x)
+    return sets
+
+
+def step_fn(wl, ops, workspace):
+    if wl.decode:
+        def step(x, stream):
+            ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
+                            lse=x["lse"], workspace=workspace, stream=stream)
+    else:
+        def step(x, stream):
+            ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
+                         lse=x["lse"], stream=stream)
+    return step
+
+
+def cpu_baseline(wl, x, budget_s):
+    """The fp64 oracle on a bounded random sample of the workload's rows (timed on
+    this host's cores).  Returns (rate, cores, description, seconds); the rate is in
+    masked TFLOP/s for prefill and in GB/s of key/value cache consumed for decode."""
+    import numpy as np
+    import torch
+    from oracle import oracle as O
+
+    g = torch.Generator().manual_seed(12345)
+    if wl.decode:
+        # Rows of decode span the whole cache: sample (sequence, key/value head)
+        # groups and copy only that group's cache slice to the host.
+        G = wl.group
+        t_all, nbytes, groups = 0.0, 0.0, 0
+        while t_all < budget_s and groups < 64:
+            b = int(torch.randint(0, wl.B, (1,), generator=g))
+            kv = int(torch.randint(0, wl.Hkv, (1,), generator=g))
+            heads = list(range(kv * G, (kv + 1) * G))
+            k_sl = x["k"][b:b + 1, :, kv:kv + 1, :].cpu()
+            v_sl = x["v"][b:b + 1, :, kv:kv + 1, :].cpu()
+            q = x["q"][b, heads].float().cpu()
+            r = x["r"][b, heads].cpu().reshape(G, 1)
+            proj = x["w"][heads].cpu().reshape(G, 1, wl.R)
+            req = np.array([(0, hl, wl.T - 1) for hl in range(G)], dtype=np.int64)
+            t0 = time.perf_counter()
+            O.attn_rows(q, r, proj, k_sl, v_sl, req, G, wl.window, wl.R, wl.scale)
+            t_all += time.perf_counter() - t0
+            nbytes += 2 * wl.attended_pairs() * wl.d * (2 if wl.dtype == "bf16" else 4)
+            groups += 1
+        return nbytes / t_all / 1e9, O.num_threads(), \
+            "%d (sequence, kv-head) groups of %s, all %d query heads each over the full cache (%.1f s)" % (
+                groups, wl.name, G, t_all), t_all
+
+    k_cpu = x["k"].cpu()
+    v_cpu = x["v"].cpu()
+    proj = x["w"].cpu().reshape(wl.Hq, 1, wl.R)
+
+    def draw(n):
+        b = torch.randint(0, wl.B, (n,), generator=g)
+        h = torch.randint(0, wl.Hq, (n,), generator=g)
+        i = torch.randint(0, wl.T, (n,), generator=g)
+        idx = [t.to(x["q"].device) for t in (b, i, h)]
+        q = x["q"][idx[0], idx[1], idx[2]].float().cpu()
+        r = x["r"][idx[0], idx[1], idx[2]].cpu()
+        rows = torch.stack([b, h, i], 1).numpy().astype(np.int64)
+        return rows, q, r.reshape(-1, 1)
+
+    def flops(rows):
+        i = rows[:, 2]
+        n = i + 1 if wl.window <= 0 else np.minimum(i + 1, wl.window)
+        return float(4 * wl.d * n.sum())
+
+    rows, q, r = draw(8)
+    O.attn_rows(q, r, proj, k_cpu, v_cpu, rows, wl.Hq, wl.window, wl.R, wl.scale)   # load, warm up
+    rows, q, r = draw(256)
+    t0 = time.perf_counter()
+    O.attn_rows(q, r, proj, k_cpu, v_cpu, rows, wl.Hq, wl.window, wl.R, wl.scale)
+    per_row = max((time.perf_counter() - t0) / len(rows), 1e-6)
+    n = int(max(8, min(4000000, budget_s / per_row)))
+    rows, q, r = draw(n)
+    t0 = time.perf_counter()
+    O.attn_rows(q, r, proj, k_cpu, v_cpu, rows, wl.Hq, wl.window, wl.R, wl.scale)
+    dt = time.perf_counter() - t0
+    return flops(rows) / dt / 1e12, O.num_threads(), \
+        "%d random (b,h,i) rows of %s (%.3g masked GFLOP, %.1f s)" % (n, wl.name, flops(rows) / 1e9, dt), dt
+
+
+def run_ours(args, wl, peaks, peaks_kind):
+    import numpy as np  # noqa: F401
+    import torch
+    import torch.distributed as dist
+    from attention_learned_relative_b200 import build, ops
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    build.build()  # no-op when the in-tree library is current
+
+    # Per-step footprint; rotate over enough input sets to exceed 3x the L2.
+    esz = 2 if wl.dtype == "bf16" else 4
+    if wl.decode:
+        step_bytes = wl.kv_bytes()
+    else:
+        step_bytes = (2 * wl.B * wl.T * wl.Hq * wl.d + 2 * wl.B * wl.T * wl.Hkv * wl.d) * esz
+    l2 = 126 * 2 ** 20
+    nsets = 1 if step_bytes > 3 * l2 else int(math.ceil(3 * l2 / step_bytes)) + 1
+    sets = make_sets(wl, nsets, dev)
+    workspace = None
+    if wl.decode:
+        nbytes = ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    step = step_fn(wl, ops, workspace)
+    stream = torch.cuda.current_stream(dev)
+
+    # Warm-up; then size the timed region to ~2 s unless --steps is given.
+    t0 = time.perf_counter()
+    for i in range(max(args.warmup, 1)):
+        step(sets[i % nsets], stream)
+    torch.cuda.synchronize()
+    warm_ms = (time.perf_counter() - t0) * 1e3 / max(args.warmup, 1)
+    steps = args.steps if args.steps is not None else int(max(20, min(20000, 2000.0 / max(warm_ms, 1e-3))))
+    ops.device_status(reset=True)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for i in range(steps):
+            step(sets[i % nsets], stream)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    status = ops.device_status(reset=True)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / steps
+
+    # End to end through the public API: pinned host inputs -> device -> kernel -> host.
+    e2e = None
+    if not args.no_e2e:
+        x = sets[0]
+        names_in = ["q", "r"] if wl.decode else ["q", "k", "v", "r", "w"]
+        host_in = {n: x[n].cpu().pin_memory() for n in names_in}
+        host_out = torch.empty(x["o"].shape, dtype=x["o"].dtype, pin_memory=True)
+        bi = sum(t.numel() * t.element_size() for t in host_in.values())
+        bo = host_out.numel() * host_out.element_size()
+        e2e_steps = max(3, min(steps, 50))
+
+        def e2e_step():
+            for n, t in host_in.items():
+                x[n].copy_(t, non_blocking=True)
+            step(x, stream)
+            host_out.copy_(x["o"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"e_ms": e_ms, "bi": bi, "bo": bo}
+
+    result = None
+    if rank == 0:
+        traffic = profile_traffic(wl.name)
+        if wl.decode:
+            unit = "GB/s"
+            per_step = wl.kv_bytes()
+            value = per_step * world / (ms_step * 1e-3) / 1e9
+            achieved = per_step / (ms_step * 1e-3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": traffic, "peak_source": peaks_kind + " hbm_gbs (copy)",
+                    "kernel": "decode_splitkv_kernel + decode_combine_kernel",
+                    "algorithmic_bytes_per_launch": per_step}
+        else:
+            unit = "TFLOP/s"
+            per_step = wl.masked_flops()
+            value = per_step * world / (ms_step * 1e-3) / 1e12
+            achieved = per_step / (ms_step * 1e-3) / 1e12
+            peak = float(peaks["bf16_tflops"])
+            if wl.dtype != "bf16":
+                # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+                peak = 148 * 128 * 2 * 1.965e9 / 1e12
+            roof = {"bound": "tensor" if wl.dtype == "bf16" else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "peak_source": (peaks_kind + " bf16_tflops (burst)") if wl.dtype == "bf16"
+                    else "fp32 FMA units x max clock",
+                    "frac_of_datasheet_2250": achieved / 2250.0,
+                    "kernel": "prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel",
+                    "algorithmic_flops_per_launch": per_step}
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": unit,
+            "n_gpus": world,
+            "steps": steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": wl.dtype,
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                       "window": wl.window, "R": wl.R, "parallelism": "dp%d (independent replicas)" % world,
+                       "l2": ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6))
+                       if nsets > 1 else "per-step input %.0f MB > L2" % (step_bytes / 1e6)},
+            "roofline": roof,
+            "clocks": clocks.summary(),
+            "gpu_launches": steps * (2 if wl.decode else 1),
+            "kernel_status": status,
+        }
+        if e2e is not None:
+            e_val = per_step * world / (e2e["e_ms"] * 1e-3) / (1e9 if wl.decode else 1e12)
+            result["e2e"] = {"value": e_val, "unit": unit, "h2d_bytes_per_step": e2e["bi"],
+                             "d2h_bytes_per_step": e2e["bo"], "ms_per_step": e2e["e_ms"]}
+        if world == 1 and not args.no_cpu_baseline:
+            v, cores, desc, _ = cpu_baseline(wl, sets[0], args.cpu_seconds)
+            result["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, wl, steps_default=5):
+    """The fp64 CPU oracle, as it stands, timed on this host's cores: each step is a
+    bounded random sample of the workload's rows (inputs drawn on the GPU when one is
+    present, else on the CPU)."""
+    import torch
+    from attention_learned_relative_b200 import workloads
+    from oracle import oracle as O
+
+    O.build()
+    steps = args.steps if args.steps is not None else steps_default
+    warm = max(args.warmup, 0)
+    per_step_s = max(0.5, min(5.0, 150.0 / max(1, steps + warm)))
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = workloads.make_inputs(wl, device=dev)
+    tot_work = 0.0
+    tot_s = 0.0
+    desc = None
+    cores = O.num_threads()
+    for s in range(warm + steps):
+        rate, cores, desc, dt = cpu_baseline(wl, x, per_step_s)
+        if s >= warm:
+            tot_work += rate * dt
+            tot_s += dt
+    value = tot_work / tot_s
+    unit = "GB/s" if wl.decode else "TFLOP/s"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": steps,
+        "warmup": warm, "ms_per_step": tot_s * 1e3 / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                   "window": wl.window, "R": wl.R},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from attention_learned_relative_b200.workloads import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    peaks, kind = load_peaks()
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+    res = run_ours(args, wl, peaks, kind)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
