@@ -256,3 +256,6 @@ extern "C" int relbias_device_status(int reset) {
 }
 
 extern "C" int relbias_version(void) { return 100; }
+
+// The allocation-free decode variant (its own file: it owns a static device array).
+#include "decode_noalloc.cu"

@@ -35,6 +35,8 @@ SIGNATURES = {
     "relbias_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ,
                                  _VP]),
+    "relbias_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                         _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_version": (_I, []),
@@ -152,6 +154,29 @@ def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | N
     rc = lib().relbias_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
                                    B, N, Hq, Hkv, d, int(window), int(R), float(scale), _dtype_code(q),
                                    _ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | None = None, out=None,
+                        lse=None, stream=None):
+    """attn_decode for callers that cannot allocate device memory: the split
+    partials go to the library's own static scratch (see
+    relbias_attn_decode_noalloc in include/relbias_attn.h for its size limit and
+    the rule that calls must not overlap on the GPU).  `out` must be given by a
+    caller that cannot allocate; None allocates it here for convenience."""
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "q [B,Hq,d], cache [B,N,Hkv,d]")
+    B, Hq, d = q.shape
+    _, N, Hkv, _ = k_cache.shape
+    for t in (q, k_cache, v_cache, r, w, out, lse):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out),
+                                           _ptr(lse), B, N, Hq, Hkv, d, int(window), int(R), float(scale),
+                                           _dtype_code(q), _stream_handle(stream, q.device))
     _check(rc)
     return out
 

@@ -58,6 +58,9 @@ extern "C" {
 #define RELBIAS_ERR_UNSUPPORTED -2  /* valid request this build or device cannot serve    */
 #define RELBIAS_ERR_CUDA        -3  /* a CUDA runtime call or kernel launch failed        */
 
+/* Bytes of the static scratch behind relbias_attn_decode_noalloc (8 MiB). */
+#define RELBIAS_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
 /* Bits of the device-side status word (relbias_device_status). */
 #define RELBIAS_STATUS_TIMEOUT   1u /* a bounded wait inside a kernel ran out             */
 
@@ -122,6 +125,35 @@ RELBIAS_API int relbias_attn_decode(const void* q, const void* k_cache, const vo
                         int B, int n_ctx, int Hq, int Hkv, int d,
                         int window, int R, float scale,
                         int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Decode that allocates nothing, for callers that cannot allocate device memory
+ * (e.g. a plugin inside an inference runtime that owns all device allocations, or
+ * a serving loop that must not call cudaMalloc/cudaFree between steps).  The
+ * paper has no counterpart; this is a property of the library, not of the method.
+ *
+ * Same arguments, results and rules as relbias_attn_decode, without the
+ * workspace: the split partials go to a scratch array of
+ * RELBIAS_DECODE_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU
+ * that loads the library holds until the process exits.
+ *   - A call whose partials need more than that (see
+ *     relbias_attn_decode_workspace_size) is rejected with RELBIAS_ERR_UNSUPPORTED
+ *     and launches nothing.
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture.
+ *   - All calls on a device share the one scratch array, which keeps the last
+ *     call's contents (every value a call reads it writes first).  Calls that
+ *     overlap on the GPU -- on different streams without ordering between them --
+ *     race on it and must not be issued.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+RELBIAS_API int relbias_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                        const float* r, const float* w,
+                        void* o, float* lse,
+                        int B, int n_ctx, int Hq, int Hkv, int d,
+                        int window, int R, float scale,
+                        int dtype, void* stream);
 
 /* Description of the last failed call on this thread ("" if none).  The string
  * stays valid until the next library call on the same thread. */
