@@ -23,6 +23,7 @@ struct PrefillParams {
     float scale_log2;        // scale * log2(e)
     float inv_scale;         // 1 / scale
 };
+int prefill_bf16_table_copies(int d, int R);   // 0 if R does not fit shared memory
 int prefill_bf16_smem_bytes(int d, int R);
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream);

@@ -10,11 +10,13 @@
 //
 // Work item: (sequence b, key/value head g, a pair of query heads of that group,
 // a 128-row query tile).  The two heads ("slots") share every K/V tile.
-// Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue of slot 0 (TMEM lanes 0-127, one row per thread)
-//   warps 4-7  softmax + epilogue of slot 1
-//   warp 8     TMA producer (Q per item, K and V per tile, 2-stage ring each)
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3   softmax + epilogue of slot 0 (TMEM lanes 0-127, one row per thread)
+//   warps 4-7   softmax + epilogue of slot 1
+//   warp 8      TMA producer (Q per item, K and V per tile, 2-stage ring each)
+//   warp 9      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle; the third warpgroup hands its registers to the softmax
+//               warpgroups (setmaxnreg), which hold a whole 128-wide row of S.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D);
 // the softmax writes P (bf16, packed in pairs) over the first 64 columns of its S.
 // MMA issue order per KV tile j:  QK0(j)  PV1(j-1)  QK1(j)  PV0(j), so one slot's
@@ -22,6 +24,14 @@
 // issue order, so QK_s(j+1) may overwrite P_s(j) once PV_s(j) has been issued, and
 // when S_s(j) is complete, O_s holds everything up to PV_s(j-1) (softmax may
 // rescale it before releasing P_s(j)).
+//
+// Bias lookup: thread t (query row i0+t) needs w[h, delta0 + t - c] for the 128
+// key columns c of a tile -- a contiguous, descending run of the table.  The table
+// is stored reversed (entry y holds w[h, Cmax - y], zero outside [0, R)), so the
+// run is ascending, in NCOPY copies shifted by one entry each: every thread picks
+// the copy that makes its run start on an NCOPY-float boundary and reads it with
+// 64- or 128-bit loads.  Copy strides are chosen so that a warp's loads hit
+// distinct banks.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -37,12 +47,20 @@ namespace {
 constexpr int kBM = 128;            // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;            // keys per tile
 constexpr int kStages = 2;          // K and V ring depth
-constexpr int kThreads = 320;
-constexpr int kPadL = 128;          // distance dd lives at table[dd + kPadL]
-constexpr int kTabExtra = 384;      // zeros around the R entries (covers -127 .. R+254)
+constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows by > 2^8
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
+constexpr int kMaxDynSmem = 232448;          // 227 KB per CTA on sm_100
 
-__host__ __device__ constexpr int tab_floats(int R) { return ((R + kTabExtra + 31) / 32) * 32; }
+// Reversed table: entry y <-> distance Cmax - y, Cmax = R + 255 (largest distance a
+// biased tile reaches is R + 254, smallest is -127).
+__host__ __device__ constexpr int tab_cmax(int R) { return R + 255; }
+__host__ __device__ constexpr int tab_len(int R) { return ((R + 392 + 31) / 32) * 32; }
+__host__ __device__ constexpr int tab_stride(int R, int ncopy) {
+    return tab_len(R) + (ncopy == 4 ? 8 : ncopy == 2 ? 18 : 0);
+}
+__host__ __device__ constexpr int tab_floats(int R, int ncopy) { return ncopy * tab_stride(R, ncopy); }
 
 template <int D>
 struct Layout {
@@ -63,6 +81,11 @@ struct Bars {
     uint32_t tmem_base;
     int abort_flag;
 };
+
+int smem_bytes_for(int d, int R, int ncopy) {
+    const int lay = d == 64 ? Layout<64>::kTab : Layout<128>::kTab;
+    return lay + 2 * tab_floats(R, ncopy) * 4 + static_cast<int>(sizeof(Bars)) + 1024;
+}
 
 struct Item {
     int qt, b, g, hp;
@@ -114,16 +137,42 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
-template <int D>
+// s[c] += rs * w[h, delta0 + t - c] for the 128 columns, from this thread's run of
+// the reversed table (`run` points at entry base_t, NCOPY-float aligned).
+template <int NCOPY>
+__device__ __forceinline__ void add_bias(float (&s)[kBN], const float* run, float rs) {
+    const uint64_t rs2 = f2_pack(rs, rs);
+#pragma unroll
+    for (int c = 0; c < kBN; c += 4) {
+        float w0, w1, w2, w3;
+        if constexpr (NCOPY == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(run + c);
+            w0 = v.x, w1 = v.y, w2 = v.z, w3 = v.w;
+        } else if constexpr (NCOPY == 2) {
+            const float2 a = *reinterpret_cast<const float2*>(run + c);
+            const float2 b = *reinterpret_cast<const float2*>(run + c + 2);
+            w0 = a.x, w1 = a.y, w2 = b.x, w3 = b.y;
+        } else {
+            w0 = run[c], w1 = run[c + 1], w2 = run[c + 2], w3 = run[c + 3];
+        }
+        const uint64_t lo = f2_fma(rs2, f2_pack(w0, w1), f2_pack(s[c], s[c + 1]));
+        const uint64_t hi = f2_fma(rs2, f2_pack(w2, w3), f2_pack(s[c + 2], s[c + 3]));
+        f2_unpack(lo, s[c], s[c + 1]);
+        f2_unpack(hi, s[c + 2], s[c + 3]);
+    }
+}
+
+template <int D, int NCOPY>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tabn = tab_floats(p.R);
+    const int tstride = tab_stride(p.R, NCOPY);
+    const int tslot = NCOPY * tstride;
     float* tables = reinterpret_cast<float*>(smem + L::kTab);
-    Bars* bars = reinterpret_cast<Bars*>(smem + L::kTab + 2 * tabn * 4);
+    Bars* bars = reinterpret_cast<Bars*>(smem + L::kTab + 2 * tslot * 4);
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -161,9 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp >= 8) {
+        regs_decrease<kOtherRegs>();
+        if (warp == 8 && lane == 0) {
+            // -------------------------------------------------------- TMA producer
             int kv_it = 0, item_it = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
@@ -194,10 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     it.g, j0, it.b);
                 }
             }
-        }
-    } else if (warp == 9) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 9 && lane == 0) {
+            // -------------------------------------------------------- MMA issuer
             const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
             const uint32_t s_tm[2] = {tmem_base, tmem_base + 128};
@@ -261,13 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ softmax / epilogue
+        regs_increase<kSoftmaxRegs>();
         const int slot = threadIdx.x >> 7;
         const int t = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
         const uint32_t s_tm = tmem_base + lane_off + slot * 128;
         const uint32_t o_tm = tmem_base + lane_off + 256 + slot * 128;
-        float* wtab = tables + slot * tabn;
+        float* wtab = tables + slot * tslot;
+        const int cmax = tab_cmax(p.R);
         const float c1 = p.scale_log2;
+        const uint64_t c1x2 = f2_pack(c1, c1);
         int tile_it = 0, item_it = 0;
         bool ok = slot < p.nslots;
         for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
@@ -277,10 +328,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             kv_range(p, i0, j_first, ntiles);
             const int h = it.g * p.G + it.hp * p.nslots + slot;
 
-            // This head's distance table, zero outside [0, R), staged once per item.
+            // This head's reversed distance table, NCOPY shifted copies, staged per item.
             named_bar_sync(1 + slot, kBM);
-            for (int x = t; x < tabn; x += kBM) {
-                const int dd = x - kPadL;
+            for (int x = t; x < tslot; x += kBM) {
+                const int cp = x / tstride;
+                const int src = x - cp * tstride + cp;
+                const int dd = cmax - src;
                 wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(p.w + static_cast<size_t>(h) * p.R + dd) : 0.0f;
             }
             named_bar_sync(1 + slot, kBM);
@@ -290,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale
                                     : 0.0f;
             float m_used = -INFINITY;   // running max, log2 units
-            float l = 0.0f;
+            uint64_t l2 = 0;            // running sum, two partial lanes (0.0f, 0.0f)
 
             for (int tt = 0; tt < ntiles; ++tt, ++tile_it) {
                 const int j0 = j_first + tt * kBN;
@@ -309,9 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (delta0 - (kBN - 1) < p.R) {
                     // Some key of this tile is closer than R: add r_i * w[h, i-j] (in units
                     // of the unscaled logit; the table is zero outside [0, R)).
-                    const float* wp = wtab + kPadL + delta0 + t;
-#pragma unroll
-                    for (int c = 0; c < kBN; ++c) s[c] = fmaf(rs, wp[-c], s[c]);
+                    const int base = cmax - delta0 - t;
+                    const int cp = base & (NCOPY - 1);
+                    add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
                 }
                 if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
                     const int hi = delta0 + t;   // causal: key c visible iff c <= hi
@@ -319,15 +372,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
                 }
-                float mx = s[0];
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-                for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+                for (int c = 4; c < kBN; c += 8) {
+                    mx0 = fmax3f(mx0, s[c], s[c + 1]);
+                    mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
+                    mx2 = fmax3f(mx2, s[c + 4], s[c + 5]);
+                    if (c + 7 < kBN) mx3 = fmax3f(mx3, s[c + 6], s[c + 7]);
+                    else mx3 = fmaxf(mx3, s[c + 6]);
+                }
+                const float mx = fmaxf(fmax3f(mx0, mx1, mx2), mx3);
                 const float m_tile = mx * c1;
                 const bool grow = m_tile > m_used + kRescaleThreshold;
                 float alpha = 1.0f;
                 if (grow) {
                     alpha = ex2_approx(m_used - m_tile);
-                    l *= alpha;
+                    l2 = f2_mul(l2, f2_pack(alpha, alpha));
                     m_used = m_tile;
                 }
                 if (tt > 0 && __any_sync(0xffffffffu, grow)) {
@@ -344,14 +404,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_wait();
                 }
                 const float mb = (m_used == -INFINITY) ? 0.0f : m_used;
+                const uint64_t nm2 = f2_pack(-mb, -mb);
                 uint32_t pk[kBN / 2];
+                uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int c = 0; c < kBN; c += 2) {
-                    const float p0 = ex2_approx(fmaf(s[c], c1, -mb));
-                    const float p1 = ex2_approx(fmaf(s[c + 1], c1, -mb));
-                    l += p0 + p1;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), c1x2, nm2), x0, x1);
+                    const float p0 = ex2_approx(x0);
+                    const float p1 = ex2_approx(x1);
+                    acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
+                l2 = f2_add(l2, f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
                 tmem_st32(s_tm, pk);
                 tmem_st32(s_tm + 32, pk + 32);
                 tmem_st_wait();
@@ -364,6 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = warp_all(mbar_wait(&bars->o_final[slot], item_it & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
+            float la, lb;
+            f2_unpack(l2, la, lb);
+            const float l = la + lb;
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
             __nv_bfloat16* orow = p.o + ((static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * D;
 #pragma unroll
@@ -395,11 +463,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+template <int D, int NCOPY>
+cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const PrefillParams& p, int smem, int grid, cudaStream_t stream) {
+    auto kern = prefill_bf16_sm100_kernel<D, NCOPY>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
+int prefill_bf16_table_copies(int d, int R) {
+    for (int nc = 4; nc >= 1; nc >>= 1)
+        if (smem_bytes_for(d, R, nc) <= kMaxDynSmem) return nc;
+    return 0;
+}
+
 int prefill_bf16_smem_bytes(int d, int R) {
-    const int lay = d == 64 ? Layout<64>::kTab : Layout<128>::kTab;
-    const int need = lay + 2 * tab_floats(R) * 4 + static_cast<int>(sizeof(Bars)) + 1024;
+    const int nc = prefill_bf16_table_copies(d, R);
+    if (nc == 0) return -1;
+    const int need = smem_bytes_for(d, R, nc);
     // Each CTA allocates all 512 TMEM columns: never let two CTAs share an SM
     // (228 KB of shared memory per SM, so more than 114 KB each).
     return need > 120 * 1024 ? need : 120 * 1024;
@@ -407,18 +492,17 @@ int prefill_bf16_smem_bytes(int d, int R) {
 
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream) {
+    const int nc = prefill_bf16_table_copies(d, p.R);
     const int smem = prefill_bf16_smem_bytes(d, p.R);
-    cudaError_t e;
+    if (nc == 0 || smem < 0) return cudaErrorInvalidValue;
     if (d == 128) {
-        e = cudaFuncSetAttribute(prefill_bf16_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        prefill_bf16_sm100_kernel<128><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
-    } else {
-        e = cudaFuncSetAttribute(prefill_bf16_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        prefill_bf16_sm100_kernel<64><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+        if (nc == 4) return launch_variant<128, 4>(tq, tk, tv, p, smem, grid, stream);
+        if (nc == 2) return launch_variant<128, 2>(tq, tk, tv, p, smem, grid, stream);
+        return launch_variant<128, 1>(tq, tk, tv, p, smem, grid, stream);
     }
-    return cudaGetLastError();
+    if (nc == 4) return launch_variant<64, 4>(tq, tk, tv, p, smem, grid, stream);
+    if (nc == 2) return launch_variant<64, 2>(tq, tk, tv, p, smem, grid, stream);
+    return launch_variant<64, 1>(tq, tk, tv, p, smem, grid, stream);
 }
 
 }  // namespace relbias

@@ -138,7 +138,8 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     }
 
     if (d != 64 && d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill supports d in {64, 128}, got %d", d);
-    if (R > 2048) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
+    if (R > 2048 || prefill_bf16_table_copies(d, R) == 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
     DeviceInfo dev;
     if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
     if (dev.major != 10 || dev.minor != 0)
