@@ -89,9 +89,8 @@ __device__ __forceinline__ uint32_t swz(int key, int dcol) {
 __global__ void __launch_bounds__(kDThreads, 1)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const DecodeParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    DecodeSmem* sm =
-        reinterpret_cast<DecodeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    DecodeSmem* sm = reinterpret_cast<DecodeSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     DecodeBars* bars = &sm->bars;
     volatile int* abort_flag = &bars->abort_flag;
 

@@ -137,6 +137,36 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
+// 2^x for a pair of fp32 values on the FMA pipe, relieving the MUFU unit (which
+// computes 16 exponentials per SM per clock against 128 FMA lanes).  Cody-Waite
+// style split x = n + f with n = round(x) (added to 1.5*2^23, whose low mantissa
+// bits then hold n) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients are a minimax fit of the relative error on that interval (7.5e-5);
+// 2^n added into the exponent field.  x is clamped below at -126.5, so exponents
+// stay in range and -inf (masked keys) gives ~5e-39 instead of 0: weights that
+// small change no sum and no bf16 P.
+constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
+                kExpC3 = 5.517166853e-02f;
+constexpr int kEmuPer8 = 3;   // of every 8 exponential pairs, this many run on the FMA pipe
+
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+    float a, b;
+    f2_unpack(x2, a, b);
+    const uint64_t xc = f2_pack(fmaxf(a, -126.5f), fmaxf(b, -126.5f));
+    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t y = f2_add(xc, magic);
+    const uint64_t n = f2_add(y, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), xc);
+    uint64_t q = f2_fma(f, f2_pack(kExpC3, kExpC3), f2_pack(kExpC2, kExpC2));
+    q = f2_fma(q, f, f2_pack(kExpC1, kExpC1));
+    q = f2_fma(q, f, f2_pack(kExpC0, kExpC0));
+    float qa, qb, ya, yb;
+    f2_unpack(q, qa, qb);
+    f2_unpack(y, ya, yb);
+    return f2_pack(__uint_as_float(__float_as_uint(qa) + (__float_as_uint(ya) << 23)),
+                   __uint_as_float(__float_as_uint(qb) + (__float_as_uint(yb) << 23)));
+}
+
 // s[c] += rs * w[h, delta0 + t - c] for the 128 columns, from this thread's run of
 // the reversed table (`run` points at entry base_t, NCOPY-float aligned).
 template <int NCOPY>
@@ -167,8 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using L = Layout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base for the 128-byte-swizzled tiles; stays a shared-space
+    // pointer, so table reads compile to shared-memory loads.
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tstride = tab_stride(p.R, NCOPY);
     const int tslot = NCOPY * tstride;
     float* tables = reinterpret_cast<float*>(smem + L::kTab);
@@ -329,12 +361,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h = it.g * p.G + it.hp * p.nslots + slot;
 
             // This head's reversed distance table, NCOPY shifted copies, staged per item.
+            // Loads are issued eight at a time so their L2 latencies overlap.
             named_bar_sync(1 + slot, kBM);
-            for (int x = t; x < tslot; x += kBM) {
-                const int cp = x / tstride;
-                const int src = x - cp * tstride + cp;
-                const int dd = cmax - src;
-                wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(p.w + static_cast<size_t>(h) * p.R + dd) : 0.0f;
+            {
+                const float* wrow = p.w + static_cast<size_t>(h) * p.R;
+                for (int x0 = 0; x0 < tslot; x0 += 8 * kBM) {
+                    float v[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int x = x0 + k * kBM + t;
+                        const int cp = x / tstride;
+                        const int dd = cmax - (x - cp * tstride + cp);
+                        v[k] = (x < tslot && dd >= 0 && dd < p.R) ? __ldg(wrow + dd) : 0.0f;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int x = x0 + k * kBM + t;
+                        if (x < tslot) wtab[x] = v[k];
+                    }
+                }
             }
             named_bar_sync(1 + slot, kBM);
 
@@ -367,10 +412,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
                 }
                 if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
-                    const int hi = delta0 + t;   // causal: key c visible iff c <= hi
+                    // Key c is visible to row t iff lo <= c <= hi.  A 32-column chunk the
+                    // whole warp sees entirely is skipped (a warp-uniform branch); other
+                    // chunks pay per-element compares.
+                    const int hi = delta0 + t;
                     const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
+                    const int t0 = t & ~31;
+                    const int hi_min = delta0 + t0;
+                    const int lo_max = p.window > 0 ? hi_min + 31 - p.window + 1 : INT_MIN;
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
+                    for (int cc = 0; cc < kBN; cc += 32) {
+                        if (!(hi_min >= cc + 31 && lo_max <= cc)) {               // not all visible
+#pragma unroll
+                            for (int c = cc; c < cc + 32; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
+                        }
+                    }
                 }
                 float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
@@ -409,10 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int c = 0; c < kBN; c += 2) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), c1x2, nm2), x0, x1);
-                    const float p0 = ex2_approx(x0);
-                    const float p1 = ex2_approx(x1);
+                    const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c1x2, nm2);
+                    float p0, p1;
+                    if (((c >> 1) & 7) < kEmuPer8) {
+                        f2_unpack(exp2_fma2(x2), p0, p1);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(x2, x0, x1);
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
                     acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
