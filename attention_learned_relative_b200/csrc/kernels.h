@@ -20,6 +20,9 @@ struct PrefillParams {
     int window, R;
     int n_qt;                // ceil(T / 128)
     int total_items;         // n_qt * B * Hkv * HP
+    int contiguous;          // 1: each CTA takes a contiguous run of items, query tiles innermost
+                             //    (sliding window: equal-cost items, the bias table is reused);
+                             // 0: items dealt round-robin, heaviest query tiles first (causal)
     float scale_log2;        // scale * log2(e)
     float inv_scale;         // 1 / scale
 };

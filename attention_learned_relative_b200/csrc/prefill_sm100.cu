@@ -73,7 +73,7 @@ struct Layout {
 };
 
 struct Bars {
-    uint64_t q_full, q_empty;
+    uint64_t q_full[2], q_empty[2];   // per slot: each slot's query tile is reloaded on its own
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_final[2];
@@ -91,11 +91,33 @@ struct Item {
     int qt, b, g, hp;
 };
 
-__device__ __forceinline__ Item decode_item(const PrefillParams& p, int u) {
+// Number of work items this CTA processes, and the k-th of them.
+__device__ __forceinline__ int items_of_cta(const PrefillParams& p) {
+    if (p.contiguous) {
+        const int per = (p.total_items + gridDim.x - 1) / gridDim.x;
+        return max(0, min(per, p.total_items - static_cast<int>(blockIdx.x) * per));
+    }
+    return (p.total_items - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
+}
+
+__device__ __forceinline__ Item item_at(const PrefillParams& p, int k) {
+    Item it;
+    if (p.contiguous) {
+        // Runs of consecutive query tiles of the same (b, g, head pair).
+        const int per = (p.total_items + gridDim.x - 1) / gridDim.x;
+        const int u = static_cast<int>(blockIdx.x) * per + k;
+        it.qt = u % p.n_qt;
+        int rem = u / p.n_qt;
+        it.hp = rem % p.HP;
+        rem /= p.HP;
+        it.g = rem % p.Hkv;
+        it.b = rem / p.Hkv;
+        return it;
+    }
+    const int u = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
     const int per_qt = p.B * p.Hkv * p.HP;
     const int qr = u / per_qt;
     int rem = u - qr * per_qt;
-    Item it;
     it.qt = p.n_qt - 1 - qr;   // heaviest query tiles first
     it.b = rem / (p.Hkv * p.HP);
     rem -= it.b * p.Hkv * p.HP;
@@ -147,7 +169,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 // small change no sum and no bf16 P.
 constexpr float kExpC0 = 9.999280572e-01f, kExpC1 = 6.932609677e-01f, kExpC2 = 2.426111251e-01f,
                 kExpC3 = 5.517166853e-02f;
-constexpr int kEmuPer8 = 3;   // of every 8 exponential pairs, this many run on the FMA pipe
+constexpr int kEmuPer8 = 2;   // of every 8 exponential pairs, this many run on the FMA pipe
 
 __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
     float a, b;
@@ -211,8 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->q_full[0], 1);
+        mbar_init(&bars->q_empty[0], 1);
+        mbar_init(&bars->q_full[1], 1);
+        mbar_init(&bars->q_empty[1], 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
@@ -246,20 +270,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_decrease<kOtherRegs>();
         if (warp == 8 && lane == 0) {
             // -------------------------------------------------------- TMA producer
-            int kv_it = 0, item_it = 0;
+            int kv_it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
-                const Item it = decode_item(p, u);
+            const int nitems = items_of_cta(p);
+            for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+                const Item it = item_at(p, item_it);
                 const int i0 = it.qt * kBM;
                 int j_first, ntiles;
                 kv_range(p, i0, j_first, ntiles);
                 const int h0 = it.g * p.G + it.hp * p.nslots;
-                if (item_it > 0 && !(ok = mbar_wait(&bars->q_empty, (item_it - 1) & 1, abort_flag))) break;
-                mbar_arrive_expect_tx(&bars->q_full, p.nslots * L::kTile);
-                for (int s = 0; s < p.nslots; ++s)
+                for (int s = 0; ok && s < p.nslots; ++s) {
+                    if (item_it > 0 && !(ok = mbar_wait(&bars->q_empty[s], (item_it - 1) & 1, abort_flag))) break;
+                    mbar_arrive_expect_tx(&bars->q_full[s], L::kTile);
                     for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full, bx * 64,
+                        tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full[s], bx * 64,
                                     h0 + s, i0, it.b);
+                }
+                if (!ok) break;
+                if (item_it + 1 < nitems) {
+                    // Warm L2 with the next item's query tiles while this item runs.
+                    const Item nx = item_at(p, item_it + 1);
+                    for (int s = 0; s < p.nslots; ++s)
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_prefetch_l2_4d(&tm_q, bx * 64, nx.g * p.G + nx.hp * p.nslots + s, nx.qt * kBM, nx.b);
+                }
                 for (int t = 0; t < ntiles; ++t, ++kv_it) {
                     const int st = kv_it & 1;
                     const uint32_t ph = (kv_it >> 1) & 1;
@@ -283,15 +317,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t s_tm[2] = {tmem_base, tmem_base + 128};
             const uint32_t o_tm[2] = {tmem_base + 256, tmem_base + 384};
             const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
-            int kv_it = 0, item_it = 0;
+            int kv_it = 0;
             uint32_t pcnt[2] = {0, 0};
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
-                const Item it = decode_item(p, u);
+            const int nitems = items_of_cta(p);
+            for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+                const Item it = item_at(p, item_it);
                 int j_first, ntiles;
                 kv_range(p, it.qt * kBM, j_first, ntiles);
-                if (!(ok = mbar_wait(&bars->q_full, item_it & 1, abort_flag))) break;
-                tc_fence_after();
                 int prev_st = 0;
                 for (int t = 0; t < ntiles; ++t, ++kv_it) {
                     const int st = kv_it & 1;
@@ -299,9 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t k_addr = smem_u32(smem + L::kK + st * L::kTile);
                     const uint32_t v_addr = smem_u32(smem + L::kV + st * L::kTile);
                     if (!(ok = mbar_wait(&bars->k_full[st], ph, abort_flag))) break;
+                    if (t == 0 && !(ok = mbar_wait(&bars->q_full[0], item_it & 1, abort_flag))) break;
                     tc_fence_after();
                     issue_qk<D>(s_tm[0], q_addr[0], k_addr, idesc_qk);
                     umma_commit(&bars->s_full[0]);
+                    if (t == ntiles - 1) umma_commit(&bars->q_empty[0]);
                     if (p.nslots == 2) {
                         if (t > 0) {
                             if (!(ok = mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag))) break;
@@ -311,11 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         t - 1 > 0);
                             umma_commit(&bars->v_empty[prev_st]);
                         }
+                        if (t == 0 && !(ok = mbar_wait(&bars->q_full[1], item_it & 1, abort_flag))) break;
+                        tc_fence_after();
                         issue_qk<D>(s_tm[1], q_addr[1], k_addr, idesc_qk);
                         umma_commit(&bars->s_full[1]);
+                        if (t == ntiles - 1) umma_commit(&bars->q_empty[1]);
                     }
                     umma_commit(&bars->k_empty[st]);
-                    if (t == ntiles - 1) umma_commit(&bars->q_empty);
                     if (!(ok = mbar_wait(&bars->v_full[st], ph, abort_flag))) break;
                     if (!(ok = mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag))) break;
                     ++pcnt[0];
@@ -351,17 +388,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cmax = tab_cmax(p.R);
         const float c1 = p.scale_log2;
         const uint64_t c1x2 = f2_pack(c1, c1);
-        int tile_it = 0, item_it = 0;
+        int tile_it = 0;
+        int staged_head = -1;
         bool ok = slot < p.nslots;
-        for (int u = blockIdx.x; ok && u < p.total_items; u += gridDim.x, ++item_it) {
-            const Item it = decode_item(p, u);
+        const int nitems = items_of_cta(p);
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const Item it = item_at(p, item_it);
             const int i0 = it.qt * kBM;
             int j_first, ntiles;
             kv_range(p, i0, j_first, ntiles);
             const int h = it.g * p.G + it.hp * p.nslots + slot;
 
-            // This head's reversed distance table, NCOPY shifted copies, staged per item.
-            // Loads are issued eight at a time so their L2 latencies overlap.
+            // This head's reversed distance table, NCOPY shifted copies, staged when the
+            // head changes.  Loads are issued eight at a time so their L2 latencies overlap.
+            if (h != staged_head) {
+            staged_head = h;
             named_bar_sync(1 + slot, kBM);
             {
                 const float* wrow = p.w + static_cast<size_t>(h) * p.R;
@@ -382,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             named_bar_sync(1 + slot, kBM);
+            }
 
             const int i = i0 + t;
             const bool row_ok = i < p.T;
@@ -428,16 +470,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+                float mc[8];
 #pragma unroll
-                for (int c = 4; c < kBN; c += 8) {
-                    mx0 = fmax3f(mx0, s[c], s[c + 1]);
-                    mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
-                    mx2 = fmax3f(mx2, s[c + 4], s[c + 5]);
-                    if (c + 7 < kBN) mx3 = fmax3f(mx3, s[c + 6], s[c + 7]);
-                    else mx3 = fmaxf(mx3, s[c + 6]);
-                }
-                const float mx = fmaxf(fmax3f(mx0, mx1, mx2), mx3);
+                for (int e = 0; e < 8; ++e) mc[e] = fmaxf(s[2 * e], s[2 * e + 1]);
+#pragma unroll
+                for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mc[e] = fmax3f(mc[e], s[c + 2 * e], s[c + 2 * e + 1]);
+                const float mx = fmaxf(fmax3f(mc[0], mc[1], mc[2]), fmax3f(fmax3f(mc[3], mc[4], mc[5]), mc[6], mc[7]));
                 const float m_tile = mx * c1;
                 const bool grow = m_tile > m_used + kRescaleThreshold;
                 float alpha = 1.0f;

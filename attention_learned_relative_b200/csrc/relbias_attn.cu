@@ -169,6 +169,7 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     const long long items = static_cast<long long>(p.n_qt) * B * Hkv * p.HP;
     if (items > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", items);
     p.total_items = static_cast<int>(items);
+    p.contiguous = p.window > 0 ? 1 : 0;
     p.scale_log2 = scale * kLog2e;
     p.inv_scale = 1.0f / scale;
     const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
