@@ -14,7 +14,8 @@
 //   warps 0-3   softmax + epilogue of slot 0 (TMEM lanes 0-127, one row per thread)
 //   warps 4-7   softmax + epilogue of slot 1
 //   warp 8      TMA producer (Q per item, K and V per tile, 2-stage ring each)
-//   warp 9      TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 9      TMEM allocator and tcgen05.mma issuer
+// The producer and MMA warps run their loops converged; one elected lane issues.
 //   warps 10-11 idle; the third warpgroup hands its registers to the softmax
 //               warpgroups (setmaxnreg), which hold a whole 128-wide row of S.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D);
@@ -137,25 +138,26 @@ __device__ __forceinline__ void kv_range(const PrefillParams& p, int i0, int& j_
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr, uint32_t idesc) {
+__device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr,
+                                         uint32_t idesc) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk & 3) * 32 + (kk >> 2) * Layout<D>::kBox;
         const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
         const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
-        umma_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+        if (leader) umma_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, uint32_t idesc,
-                                         bool accumulate) {
+__device__ __forceinline__ void issue_pv(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         uint32_t idesc, bool accumulate) {
 #pragma unroll
     for (int kk = 0; kk < kBN / 16; ++kk) {
         // V tile: keys are the K dimension (8-row groups 1024 B apart), head dim
         // is the N dimension (64-column TMA boxes kBox apart): MN-major operand.
         const uint64_t b = smem_desc_sw128(v_addr + kk * 16 * 128, Layout<D>::kBox, 1024);
-        umma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+        if (leader) umma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
     }
 }
 
@@ -268,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp >= 8) {
         regs_decrease<kOtherRegs>();
-        if (warp == 8 && lane == 0) {
+        if (warp == 8) {
             // -------------------------------------------------------- TMA producer
+            const bool leader = elect_one();
             int kv_it = 0;
             bool ok = true;
             const int nitems = items_of_cta(p);
@@ -280,14 +283,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kv_range(p, i0, j_first, ntiles);
                 const int h0 = it.g * p.G + it.hp * p.nslots;
                 for (int s = 0; ok && s < p.nslots; ++s) {
-                    if (item_it > 0 && !(ok = mbar_wait(&bars->q_empty[s], (item_it - 1) & 1, abort_flag))) break;
-                    mbar_arrive_expect_tx(&bars->q_full[s], L::kTile);
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full[s], bx * 64,
-                                    h0 + s, i0, it.b);
+                    if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->q_empty[s], (item_it - 1) & 1, abort_flag))))
+                        break;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&bars->q_full[s], L::kTile);
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full[s],
+                                        bx * 64, h0 + s, i0, it.b);
+                    }
                 }
                 if (!ok) break;
-                if (item_it + 1 < nitems) {
+                if (leader && item_it + 1 < nitems) {
                     // Warm L2 with the next item's query tiles while this item runs.
                     const Item nx = item_at(p, item_it + 1);
                     for (int s = 0; s < p.nslots; ++s)
@@ -298,20 +304,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int st = kv_it & 1;
                     const uint32_t ph = (kv_it >> 1) & 1;
                     const int j0 = j_first + t * kBN;
-                    if (!(ok = mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag))) break;
-                    mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st], bx * 64,
-                                    it.g, j0, it.b);
-                    if (!(ok = mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag))) break;
-                    mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st], bx * 64,
-                                    it.g, j0, it.b);
+                    if (!(ok = warp_all(mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag)))) break;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st],
+                                        bx * 64, it.g, j0, it.b);
+                    }
+                    if (!(ok = warp_all(mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag)))) break;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st],
+                                        bx * 64, it.g, j0, it.b);
+                    }
                 }
             }
-        } else if (warp == 9 && lane == 0) {
+        } else if (warp == 9) {
             // -------------------------------------------------------- MMA issuer
+            const bool leader = elect_one();
             const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
             const uint32_t s_tm[2] = {tmem_base, tmem_base + 128};
@@ -331,48 +342,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (kv_it >> 1) & 1;
                     const uint32_t k_addr = smem_u32(smem + L::kK + st * L::kTile);
                     const uint32_t v_addr = smem_u32(smem + L::kV + st * L::kTile);
-                    if (!(ok = mbar_wait(&bars->k_full[st], ph, abort_flag))) break;
-                    if (t == 0 && !(ok = mbar_wait(&bars->q_full[0], item_it & 1, abort_flag))) break;
+                    if (!(ok = warp_all(mbar_wait(&bars->k_full[st], ph, abort_flag)))) break;
+                    if (t == 0 && !(ok = warp_all(mbar_wait(&bars->q_full[0], item_it & 1, abort_flag)))) break;
                     tc_fence_after();
-                    issue_qk<D>(s_tm[0], q_addr[0], k_addr, idesc_qk);
-                    umma_commit(&bars->s_full[0]);
-                    if (t == ntiles - 1) umma_commit(&bars->q_empty[0]);
+                    issue_qk<D>(leader, s_tm[0], q_addr[0], k_addr, idesc_qk);
+                    if (leader) umma_commit(&bars->s_full[0]);
+                    if (leader && t == ntiles - 1) umma_commit(&bars->q_empty[0]);
                     if (p.nslots == 2) {
                         if (t > 0) {
-                            if (!(ok = mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag))) break;
+                            if (!(ok = warp_all(mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag)))) break;
                             ++pcnt[1];
                             tc_fence_after();
-                            issue_pv<D>(o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv,
-                                        t - 1 > 0);
-                            umma_commit(&bars->v_empty[prev_st]);
+                            issue_pv<D>(leader, o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile),
+                                        idesc_pv, t - 1 > 0);
+                            if (leader) umma_commit(&bars->v_empty[prev_st]);
                         }
-                        if (t == 0 && !(ok = mbar_wait(&bars->q_full[1], item_it & 1, abort_flag))) break;
+                        if (t == 0 && !(ok = warp_all(mbar_wait(&bars->q_full[1], item_it & 1, abort_flag)))) break;
                         tc_fence_after();
-                        issue_qk<D>(s_tm[1], q_addr[1], k_addr, idesc_qk);
-                        umma_commit(&bars->s_full[1]);
-                        if (t == ntiles - 1) umma_commit(&bars->q_empty[1]);
+                        issue_qk<D>(leader, s_tm[1], q_addr[1], k_addr, idesc_qk);
+                        if (leader) umma_commit(&bars->s_full[1]);
+                        if (leader && t == ntiles - 1) umma_commit(&bars->q_empty[1]);
                     }
-                    umma_commit(&bars->k_empty[st]);
-                    if (!(ok = mbar_wait(&bars->v_full[st], ph, abort_flag))) break;
-                    if (!(ok = mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag))) break;
+                    if (leader) umma_commit(&bars->k_empty[st]);
+                    if (!(ok = warp_all(mbar_wait(&bars->v_full[st], ph, abort_flag)))) break;
+                    if (!(ok = warp_all(mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag)))) break;
                     ++pcnt[0];
                     tc_fence_after();
-                    issue_pv<D>(o_tm[0], s_tm[0], v_addr, idesc_pv, t > 0);
-                    if (p.nslots == 1) umma_commit(&bars->v_empty[st]);
-                    if (t == ntiles - 1) umma_commit(&bars->o_final[0]);
+                    issue_pv<D>(leader, o_tm[0], s_tm[0], v_addr, idesc_pv, t > 0);
+                    if (leader && p.nslots == 1) umma_commit(&bars->v_empty[st]);
+                    if (leader && t == ntiles - 1) umma_commit(&bars->o_final[0]);
                     prev_st = st;
                 }
                 if (ok && p.nslots == 2) {
-                    if (!(ok = mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag))) break;
+                    if (!(ok = warp_all(mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag)))) break;
                     ++pcnt[1];
                     tc_fence_after();
-                    issue_pv<D>(o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv, ntiles > 1);
-                    umma_commit(&bars->v_empty[prev_st]);
-                    umma_commit(&bars->o_final[1]);
+                    issue_pv<D>(leader, o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv,
+                                ntiles > 1);
+                    if (leader) umma_commit(&bars->v_empty[prev_st]);
+                    if (leader) umma_commit(&bars->o_final[1]);
                 }
             }
             // Drain: wait (bounded, regardless of abort) until every MMA issued has finished.
-            umma_commit(&bars->mma_done);
+            if (leader) umma_commit(&bars->mma_done);
             int dummy = 0;
             mbar_wait(&bars->mma_done, 0, &dummy);
         }
