@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->p_full[s], kBM);
+            mbar_init(&bars->p_full[s], kBM / 32);   // one arrival per softmax warp of the slot
             mbar_init(&bars->o_final[s], 1);
         }
         mbar_init(&bars->mma_done, 1);
@@ -535,7 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st32(s_tm + 32, pk + 32);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full[slot]);
+                // One arrival per warp, once every lane's P is in tensor memory.
+                __syncwarp();
+                if ((t & 31) == 0) mbar_arrive(&bars->p_full[slot]);
             }
             if (!ok) break;
 
