@@ -20,6 +20,7 @@ struct PrefillParams {
     int window, R;
     int n_qt;                // ceil(T / 128)
     int total_items;         // n_qt * B * Hkv * HP
+    int o_v8;                // 1: o is 32-byte aligned (rows are written with 32-byte stores)
     int contiguous;          // 1: each CTA takes a contiguous run of items, query tiles innermost
                              //    (sliding window: equal-cost items, the bias table is reused);
                              // 0: items dealt round-robin, heaviest query tiles first (causal)

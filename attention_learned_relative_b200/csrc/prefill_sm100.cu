@@ -560,10 +560,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 16; ++e)
                     packed[e] = pack_bf16x2(__uint_as_float(ob[2 * e]) * inv_l, __uint_as_float(ob[2 * e + 1]) * inv_l);
                 if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
+                    // Each thread writes its own row: 32-byte stores when O allows them
+                    // (whole sectors, half the store instructions), else 16-byte ones.
+                    if (p.o_v8) {
+                        st_global_v8(orow + c, packed);
+                        st_global_v8(orow + c + 16, packed + 8);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                    }
                 }
             }
             if (p.lse != nullptr && row_ok)

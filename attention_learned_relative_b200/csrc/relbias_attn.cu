@@ -170,6 +170,7 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     if (items > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", items);
     p.total_items = static_cast<int>(items);
     p.contiguous = p.window > 0 ? 1 : 0;
+    p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
     p.scale_log2 = scale * kLog2e;
     p.inv_scale = 1.0f / scale;
     const int grid = static_cast<int>(std::min<long long>(items, dev.sms));

@@ -144,6 +144,19 @@ def test_output_buffers_fully_written():
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
 
 
+def test_output_alignment_paths_agree():
+    """O 32-byte aligned (written with 32-byte stores) and O only 16-byte aligned (16-byte
+    stores) give bit-identical results, rows of a ragged last tile included."""
+    x = _inputs(2, 333, 8, 2, 128, 128, seed=31)
+    o_a = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], 0, 128, 0.09)
+    flat = torch.empty(x["q"].numel() + 8, dtype=x["q"].dtype, device="cuda")
+    o_u = flat[8:].view(x["q"].shape)              # 16 bytes past a 256-byte aligned base
+    assert o_a.data_ptr() % 32 == 0 and o_u.data_ptr() % 32 == 16
+    ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], 0, 128, 0.09, out=o_u)
+    torch.cuda.synchronize()
+    assert torch.equal(o_a, o_u)
+
+
 def _sampled_check(wl, per_head, seed):
     x = make_inputs(wl, device="cuda")
     B, T, Hq, d = x["q"].shape
