@@ -50,7 +50,7 @@ def _load():
         f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                       ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                      ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                      ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int64,
                       ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -69,11 +69,13 @@ def _f32(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
 
 
-def attn_rows(q_rows, rs_rows, proj, k, v, req, Hq: int, window: int, R: int, scale: float):
+def attn_rows(q_rows, rs_rows, proj, k, v, req, Hq: int, window: int, R: int, scale: float, temp_n0: int = 0):
     """Rows of biased attention.
 
     q_rows [n, d], rs_rows [n, C], proj [Hp, C, R] with Hp in {1, Hq},
     k, v [B, T, Hkv, d], req [n, 3] int64 of (b, h, i), Hq query heads.
+    temp_n0 > 1 applies the context-length temperature tau(n) = max(1, ln n / ln temp_n0)
+    to the logits of a row that sees n keys (relbias_oracle.c states the reading).
     Returns (o [n, d] float64, lse [n] float64).
     """
     lib = _load()
@@ -92,10 +94,10 @@ def attn_rows(q_rows, rs_rows, proj, k, v, req, Hq: int, window: int, R: int, sc
         raise ValueError("table length %d != R %d" % (Rt, R))
     if q_rows.shape != (n, d) or rs_rows.shape != (n, C):
         raise ValueError("q_rows / rs_rows shape mismatch")
-    return _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale)
+    return _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale, temp_n0)
 
 
-def _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale):
+def _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale, temp_n0=0):
     n = req.shape[0]
     Hp, C, _ = proj.shape
     o = np.zeros((n, d), dtype=np.float64)
@@ -104,7 +106,7 @@ def _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, 
         return o, lse
     rc = lib.oracle_attn_rows(q_rows.ctypes.data, rs_rows.ctypes.data, proj.ctypes.data, Hp, C,
                               k.ctypes.data, v.ctypes.data, req.ctypes.data, n,
-                              B, T, Hq, Hkv, d, int(window), int(R), float(scale),
+                              B, T, Hq, Hkv, d, int(window), int(R), float(scale), int(temp_n0),
                               o.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError("oracle_attn_rows rejected its arguments")
@@ -123,12 +125,13 @@ def _tables(w, Hq: int, R: int) -> np.ndarray:
     raise ValueError("unsupported table shape %s for Hq=%d R=%d" % (w.shape, Hq, R))
 
 
-def attn_prefill(q, k, v, r, w, window: int, R: int, scale: float, rows=None):
+def attn_prefill(q, k, v, r, w, window: int, R: int, scale: float, rows=None, temp_n0: int = 0):
     """Causal biased attention over whole sequences.
 
     q [B, T, Hq, d]; k, v [B, T, Hkv, d]; r [B, T, Hq] (rank 1) or [B, T, Hq, C];
     w [Hq, R] (rank 1, per head) or a bank [C, R] / [1, C, R] / [Hq, C, R].
     rows: None for every (b, h, i); else an [n, 3] array of (b, h, i).
+    temp_n0: context-length temperature break point (see attn_rows); 0 = none.
     Returns (O [B, T, Hq, d], LSE [B, Hq, T]) in float64 for rows=None,
     else (o [n, d], lse [n]).
     """
@@ -156,17 +159,18 @@ def attn_prefill(q, k, v, r, w, window: int, R: int, scale: float, rows=None):
             raise ValueError("row request out of range: %s" % (req[bad][0].tolist(),))
     q_rows = np.ascontiguousarray(q[req[:, 0], req[:, 2], req[:, 1], :])
     rs_rows = np.ascontiguousarray(rs[req[:, 0], req[:, 2], req[:, 1], :])
-    o, lse = _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale)
+    o, lse = _rows_call(lib, q_rows, rs_rows, proj, k, v, req, B, T, Hq, Hkv, d, window, R, scale, temp_n0)
     if rows is not None:
         return o, lse
     return o.reshape(B, T, Hq, d), lse.reshape(B, T, Hq).transpose(0, 2, 1).copy()
 
 
-def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float):
+def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float, temp_n0: int = 0):
     """One new query per sequence at position n_ctx-1 against a cache of n_ctx rows
     that already holds the query's own key and value in its last row.
 
     q [B, Hq, d]; k_cache, v_cache [B, n_ctx, Hkv, d]; r [B, Hq] or [B, Hq, C].
+    temp_n0: context-length temperature break point (see attn_rows); 0 = none.
     Returns (O [B, Hq, d], LSE [B, Hq]) in float64.
     """
     lib = _load()
@@ -185,7 +189,7 @@ def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float):
     b_i, h_i = np.meshgrid(np.arange(B), np.arange(Hq), indexing="ij")
     req = np.stack([b_i.ravel(), h_i.ravel(), np.full(B * Hq, N - 1)], axis=1).astype(np.int64)
     o, lse = _rows_call(lib, q.reshape(B * Hq, d), r.reshape(B * Hq, C), proj, k, v, req,
-                        B, N, Hq, Hkv, d, window, R, scale)
+                        B, N, Hq, Hkv, d, window, R, scale, temp_n0)
     return o.reshape(B, Hq, d), lse.reshape(B, Hq)
 
 

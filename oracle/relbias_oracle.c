@@ -32,6 +32,15 @@
  *   layers from the concepts page, "Hybrid Attention Interaction"):
  *     A_i = { j : 0 <= i-j  and  (window <= 0 or i-j < window) }.
  *
+ *   Context-length temperature (optional; the essay, section "The temperature
+ *   scale is dependent on context length"): global layers multiply both the
+ *   query (hence the content logit) and the position bias by tau(n), n = the
+ *   number of keys the query can see, flat up to 128k tokens and growing
+ *   logarithmically beyond.  The page's formula lost its symbols; the reading
+ *   taken is the log-n scaling it names, tau(n) = max(1, ln n / ln n0), with
+ *   the break point n0 a parameter (131072 on the page; n0 <= 0 turns the
+ *   temperature off).  So the logit is tau(|A_i|) * (scale*q.k + bias).
+ *
  *   Softmax in fp64: m = max logit, O_i = sum_j exp(l_j - m) v_j / sum exp(l - m),
  *   LSE_i = m + log(sum_j exp(l_j - m)).
  *
@@ -60,7 +69,7 @@
  */
 static int oracle_row(const float* q, const float* rs, const float* proj, int C,
                       const float* k, const float* v, int64_t kv_stride,
-                      int64_t i, int64_t window, int64_t R, double scale, int d,
+                      int64_t i, int64_t window, int64_t R, double scale, int64_t temp_n0, int d,
                       double* out, double* lse)
 {
     /* step 2: the token's personal curve over distances 0..R-1 */
@@ -79,6 +88,9 @@ static int oracle_row(const float* q, const float* rs, const float* proj, int C,
     int64_t j_lo = 0;
     if (window > 0 && i - window + 1 > 0) j_lo = i - window + 1;
     int64_t n = i - j_lo + 1;
+    /* context-length temperature: tau(n) = max(1, ln n / ln n0) */
+    double tau = 1.0;
+    if (temp_n0 > 1 && n > temp_n0) tau = log((double)n) / log((double)temp_n0);
     double* logit = (double*)malloc((size_t)n * sizeof(double));
     if (!logit) { free(curve); return -1; }
 
@@ -94,8 +106,8 @@ static int oracle_row(const float* q, const float* rs, const float* proj, int C,
             int64_t idx = dist < 0 ? 0 : (dist > R - 1 ? R - 1 : dist);
             bias = (dist < 0 || dist >= R) ? 0.0 : curve[idx];
         }
-        /* step 5: add to the scaled logit */
-        double l = scale * dot + bias;
+        /* step 5: add to the scaled logit (then the temperature, if any) */
+        double l = tau * (scale * dot + bias);
         logit[j - j_lo] = l;
         if (l > m) m = l;
     }
@@ -125,6 +137,7 @@ static int oracle_row(const float* q, const float* rs, const float* proj, int C,
  *   req    [n, 3]        (b, h, i) of each requested row
  *   Hq, Hkv              query heads and key/value heads; head h reads
  *                        key/value head h / (Hq / Hkv)
+ *   temp_n0              temperature break point (<= 1: no temperature)
  *   o_out  [n, d], lse_out [n]
  * Returns 0 on success, -1 on a bad argument or allocation failure.
  */
@@ -133,7 +146,7 @@ int oracle_attn_rows(const float* q_rows, const float* rs_rows,
                      const float* k, const float* v,
                      const int64_t* req, int64_t n,
                      int B, int64_t T, int Hq, int Hkv, int d,
-                     int64_t window, int64_t R, double scale,
+                     int64_t window, int64_t R, double scale, int64_t temp_n0,
                      double* o_out, double* lse_out)
 {
     if (n < 0 || B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || C <= 0 || R < 0)
@@ -155,7 +168,7 @@ int oracle_attn_rows(const float* q_rows, const float* rs_rows,
         const float* vb = v + ((b * T) * Hkv + g) * (int64_t)d;
         const float* table = proj + (Hp == 1 ? 0 : h) * (int64_t)C * R;
         int rc = oracle_row(q_rows + u * (int64_t)d, rs_rows + u * (int64_t)C, table, C,
-                            kb, vb, (int64_t)Hkv * d, i, window, R, scale, d,
+                            kb, vb, (int64_t)Hkv * d, i, window, R, scale, temp_n0, d,
                             o_out + u * (int64_t)d, lse_out + u);
         if (rc != 0) {
 #pragma omp atomic write

@@ -337,3 +337,61 @@ def test_rejects_bad_arguments(oracle):
     with pytest.raises(ValueError):   # row index past the end
         oracle.attn_prefill(torch.zeros(1, 4, 2, 2), k, k, torch.zeros(1, 4, 2), torch.zeros(2, 2), 0, 2, 1.0,
                             rows=[(0, 0, 4)])
+
+
+# --- context-length temperature (the essay's "The temperature scale is dependent on
+# context length" section; reading: tau(n) = max(1, ln n / ln n0), n = keys the query sees)
+
+
+def test_temperature_off_is_identity(oracle):
+    """No break point, or a break point no row's key count exceeds, changes nothing."""
+    B, T, Hq, Hkv, d, R = 1, 70, 4, 2, 8, 16
+    q, k, v = (_rand(s, 150 + i).float() for i, s in enumerate([(B, T, Hq, d), (B, T, Hkv, d), (B, T, Hkv, d)]))
+    r, w = _rand((B, T, Hq), 153).float(), _rand((Hq, R), 154).float()
+    for window in (0, 32):
+        o0, l0 = oracle.attn_prefill(q, k, v, r, w, window, R, 0.3)
+        for n0 in (1, T, T + 5):
+            o1, l1 = oracle.attn_prefill(q, k, v, r, w, window, R, 0.3, temp_n0=n0)
+            np.testing.assert_array_equal(o1, o0)
+            np.testing.assert_array_equal(l1, l0)
+
+
+def test_temperature_at_square_of_break_point_doubles_logits(oracle):
+    """A row that sees n0^2 keys has tau = 2: the same as doubling both the scale and
+    the bias table without a temperature (the page scales the queries and the bias)."""
+    B, T, Hq, Hkv, d, R, n0 = 1, 90, 4, 2, 8, 24, 8
+    q, k, v = (_rand(s, 160 + i).float() for i, s in enumerate([(B, T, Hq, d), (B, T, Hkv, d), (B, T, Hkv, d)]))
+    r, w = _rand((B, T, Hq), 163).float(), _rand((Hq, R), 164).float()
+    # causal: row 63 sees exactly 64 keys; window 64: every row from 63 on does
+    for window, rows_i in ((0, [63]), (64, list(range(63, T)))):
+        rows = [(0, h, i) for h in range(Hq) for i in rows_i]
+        o_t, l_t = oracle.attn_prefill(q, k, v, r, w, window, R, 0.3, rows=rows, temp_n0=n0)
+        o_2, l_2 = oracle.attn_prefill(q, k, v, r, 2 * w, window, R, 0.6, rows=rows)
+        np.testing.assert_allclose(o_t, o_2, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(l_t, l_2, rtol=1e-12, atol=1e-12)
+
+
+def test_temperature_without_bias_is_sdpa_with_scaled_queries(oracle):
+    """With r = 0 the temperature multiplies each query row: torch SDPA on q * tau_i."""
+    B, T, Hq, Hkv, d, R, n0 = 2, 100, 4, 2, 16, 8, 16
+    q, k, v = _rand((B, T, Hq, d), 170), _rand((B, T, Hkv, d), 171), _rand((B, T, Hkv, d), 172)
+    r = torch.zeros(B, T, Hq, dtype=torch.float64)
+    w = _rand((Hq, R), 173)
+    for window in (0, 40):
+        n = torch.tensor([len(_attended(i, window)) for i in range(T)], dtype=torch.float64)
+        tau = torch.clamp(torch.log(n) / math.log(n0), min=1.0)
+        # the oracle reads float32 inputs: give SDPA the same values
+        qf, kf, vf = (x.float().double() for x in (q, k, v))
+        ref = _sdpa(qf * tau[None, :, None, None], kf, vf, 0.25, window)
+        o, _ = oracle.attn_prefill(qf, kf, vf, r, w, window, R, 0.25, temp_n0=n0)
+        np.testing.assert_allclose(o, ref.numpy(), rtol=1e-10, atol=1e-10)
+
+
+def test_temperature_decode_matches_prefill_row(oracle):
+    B, N, Hq, Hkv, d, R, n0 = 2, 60, 4, 2, 8, 12, 10
+    q, k, v = (_rand(s, 180 + i).float() for i, s in enumerate([(B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, d)]))
+    r, w = _rand((B, N, Hq), 183).float(), _rand((Hq, R), 184).float()
+    o, lse = oracle.attn_prefill(q, k, v, r, w, 0, R, 0.3, temp_n0=n0)
+    od, ld = oracle.attn_decode(q[:, -1], k, v, r[:, -1], w, 0, R, 0.3, temp_n0=n0)
+    np.testing.assert_array_equal(od, o[:, -1])
+    np.testing.assert_array_equal(ld, lse[:, :, -1])
