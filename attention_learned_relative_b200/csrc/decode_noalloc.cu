@@ -55,7 +55,8 @@ int noalloc_scratch(void** out) {
 
 extern "C" int relbias_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const float* r,
                                            const float* w, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv,
-                                           int d, int window, int R, float scale, int dtype, void* stream) {
+                                           int d, int window, int R, float scale, int temp_n0, int dtype,
+                                           void* stream) {
     using namespace relbias;
     t_err.clear();
     // Argument errors first, exactly as the regular entry point reports them.
@@ -63,7 +64,7 @@ extern "C" int relbias_attn_decode_noalloc(const void* q, const void* k_cache, c
     if (rc != RELBIAS_OK) return rc;
     if (B == 0)
         return relbias_attn_decode(q, k_cache, v_cache, r, w, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale,
-                                   dtype, nullptr, 0, stream);
+                                   temp_n0, dtype, nullptr, 0, stream);
     void* ws = nullptr;
     if ((rc = noalloc_scratch(&ws)) != RELBIAS_OK) return rc;
     const size_t need = relbias_attn_decode_workspace_size(B, Hq, Hkv, n_ctx, d, window);
@@ -73,6 +74,6 @@ extern "C" int relbias_attn_decode_noalloc(const void* q, const void* k_cache, c
                     "relbias_attn_decode_noalloc; call relbias_attn_decode with a workspace instead",
                     need, kNoAllocScratchBytes);
     // The split partials are written before they are read: nothing needs clearing.
-    return relbias_attn_decode(q, k_cache, v_cache, r, w, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale, dtype, ws,
-                               kNoAllocScratchBytes, stream);
+    return relbias_attn_decode(q, k_cache, v_cache, r, w, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale, temp_n0,
+                               dtype, ws, kNoAllocScratchBytes, stream);
 }

@@ -26,6 +26,8 @@ struct PrefillParams {
                              // 0: items dealt round-robin, heaviest query tiles first (causal)
     float scale_log2;        // scale * log2(e)
     float inv_scale;         // 1 / scale
+    int temp_n0;             // > 1: logits of a row seeing n > temp_n0 keys are scaled by ln n / ln temp_n0
+    float inv_log_n0;        // 1 / ln(temp_n0)
 };
 int prefill_bf16_table_copies(int d, int R);   // 0 if R does not fit shared memory
 int prefill_bf16_smem_bytes(int d, int R);
@@ -35,7 +37,7 @@ cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& 
 // fp32 SIMT prefill (prefill_fp32.cu).
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
                                 float* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, cudaStream_t stream);
+                                float scale, int temp_n0, cudaStream_t stream);
 
 // bf16 split-KV decode + log-sum-exp combine (decode_sm100.cu).
 struct DecodeParams {

@@ -25,7 +25,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreadsF32)
     prefill_fp32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                         const float* __restrict__ r, const float* __restrict__ w, float* __restrict__ o,
-                        float* __restrict__ lse, int T, int Hq, int Hkv, int window, int R, float scale) {
+                        float* __restrict__ lse, int T, int Hq, int Hkv, int window, int R, float scale,
+                        int temp_n0) {
     constexpr int BK = D <= 128 ? 32 : 16;   // keys per shared-memory tile
     constexpr int DL = D / 4;                 // dims per lane
     __shared__ __align__(16) float ks[BK * D];
@@ -45,7 +46,15 @@ __global__ void __launch_bounds__(kThreadsF32)
         qv[u] = row_ok ? qrow[4 * u + qd] : 0.0f;
         ov[u] = 0.0f;
     }
-    const float ri = row_ok ? r[(static_cast<size_t>(b) * T + i) * Hq + h] : 0.0f;
+    // Context-length temperature: a row that sees n > temp_n0 keys has both logit
+    // terms scaled by ln n / ln temp_n0.
+    float tau = 1.0f;
+    if (temp_n0 > 1) {
+        const int n = window > 0 ? min(i + 1, window) : i + 1;
+        if (n > temp_n0) tau = static_cast<float>(log(static_cast<double>(n)) / log(static_cast<double>(temp_n0)));
+    }
+    const float ri = row_ok ? tau * r[(static_cast<size_t>(b) * T + i) * Hq + h] : 0.0f;
+    const float scale_row = tau * scale;
     float m = -INFINITY, l = 0.0f;
 
     int j_begin = 0;
@@ -81,7 +90,7 @@ __global__ void __launch_bounds__(kThreadsF32)
             const bool valid = row_ok && j < T && dist >= 0 && (window <= 0 || dist < window);
             float x = -INFINITY;
             if (valid) {
-                x = part * scale;
+                x = part * scale_row;
                 if (dist < R) x = fmaf(ri, __ldg(w + static_cast<size_t>(h) * R + dist), x);
             }
             s[jj] = x;
@@ -114,9 +123,11 @@ __global__ void __launch_bounds__(kThreadsF32)
 
 template <int D>
 cudaError_t launch(const float* q, const float* k, const float* v, const float* r, const float* w, float* o,
-                   float* lse, int B, int T, int Hq, int Hkv, int window, int R, float scale, cudaStream_t st) {
+                   float* lse, int B, int T, int Hq, int Hkv, int window, int R, float scale, int temp_n0,
+                   cudaStream_t st) {
     dim3 grid((T + kRows - 1) / kRows, Hq, B);
-    prefill_fp32_kernel<D><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, Hq, Hkv, window, R, scale);
+    prefill_fp32_kernel<D><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, Hq, Hkv, window, R, scale,
+                                                         temp_n0);
     return cudaGetLastError();
 }
 
@@ -124,12 +135,12 @@ cudaError_t launch(const float* q, const float* k, const float* v, const float* 
 
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
                                 float* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, cudaStream_t stream) {
+                                float scale, int temp_n0, cudaStream_t stream) {
     switch (d) {
-        case 32: return launch<32>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, stream);
-        case 64: return launch<64>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, stream);
-        case 128: return launch<128>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, stream);
-        case 256: return launch<256>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, stream);
+        case 32: return launch<32>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
+        case 64: return launch<64>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
+        case 128: return launch<128>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
+        case 256: return launch<256>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
         default: return cudaErrorInvalidValue;
     }
 }

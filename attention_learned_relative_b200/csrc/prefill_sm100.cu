@@ -398,8 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_tm = tmem_base + lane_off + 256 + slot * 128;
         float* wtab = tables + slot * tslot;
         const int cmax = tab_cmax(p.R);
-        const float c1 = p.scale_log2;
-        const uint64_t c1x2 = f2_pack(c1, c1);
         int tile_it = 0;
         int staged_head = -1;
         bool ok = slot < p.nslots;
@@ -443,6 +441,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     : 0.0f;
             float m_used = -INFINITY;   // running max, log2 units
             uint64_t l2 = 0;            // running sum, two partial lanes (0.0f, 0.0f)
+            // Logit scale of this row, log2 units, with the context-length temperature:
+            // a row that sees n > temp_n0 keys has its logits (content and bias) scaled
+            // by ln n / ln temp_n0 (the essay, "The temperature scale is dependent on
+            // context length").
+            float c1 = p.scale_log2;
+            if (p.temp_n0 > 1) {
+                const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
+                if (n > p.temp_n0) c1 *= __logf(static_cast<float>(n)) * p.inv_log_n0;
+            }
+            const uint64_t c1x2 = f2_pack(c1, c1);
 
             for (int tt = 0; tt < ntiles; ++tt, ++tile_it) {
                 const int j0 = j_first + tt * kBN;

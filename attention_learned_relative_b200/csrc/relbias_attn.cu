@@ -116,7 +116,7 @@ using namespace relbias;
 
 extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, const float* r, const float* w,
                                 void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, int dtype, void* stream) {
+                                float scale, int temp_n0, int dtype, void* stream) {
     t_err.clear();
     int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
@@ -133,7 +133,7 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
             return fail(RELBIAS_ERR_UNSUPPORTED, "fp32 prefill supports d in {32, 64, 128, 256}, got %d", d);
         cudaError_t e = launch_prefill_fp32(static_cast<const float*>(q), static_cast<const float*>(k),
                                             static_cast<const float*>(v), r, w, static_cast<float*>(o), lse, B, T,
-                                            Hq, Hkv, d, window, R, scale, st);
+                                            Hq, Hkv, d, window, R, scale, temp_n0, st);
         return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "fp32 prefill launch");
     }
 
@@ -173,6 +173,8 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
     p.scale_log2 = scale * kLog2e;
     p.inv_scale = 1.0f / scale;
+    p.temp_n0 = temp_n0 > 1 ? temp_n0 : 0;
+    p.inv_log_n0 = temp_n0 > 1 ? static_cast<float>(1.0 / std::log(static_cast<double>(temp_n0))) : 0.0f;
     const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
     cudaError_t e = launch_prefill_bf16_sm100(tq, tk, tv, p, d, grid, st);
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "bf16 prefill launch");
@@ -188,8 +190,8 @@ extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int
 
 extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const void* v_cache, const float* r,
                                    const float* w, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d,
-                                   int window, int R, float scale, int dtype, void* workspace, size_t ws_bytes,
-                                   void* stream) {
+                                   int window, int R, float scale, int temp_n0, int dtype, void* workspace,
+                                   size_t ws_bytes, void* stream) {
     t_err.clear();
     int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
@@ -230,6 +232,16 @@ extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const voi
     p.chunks_per_split = (p.nchunks + p.nsplit - 1) / p.nsplit;
     p.scale_log2 = scale * kLog2e;
     p.inv_scale = 1.0f / scale;
+    {
+        // Context-length temperature of the one query row, which sees n keys: both
+        // logit terms scale by ln n / ln temp_n0 (the bias is added in units of the
+        // unscaled logit, so scaling the log2 factor scales both).
+        const int n = p.window > 0 ? std::min(n_ctx, p.window) : n_ctx;
+        if (temp_n0 > 1 && n > temp_n0)
+            p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
+                                              (std::log(static_cast<double>(n)) /
+                                               std::log(static_cast<double>(temp_n0))));
+    }
     const size_t need = decode_workspace_bytes(B, Hq, p.nsplit, d);
     if (ws_bytes < need)
         return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes, need);
@@ -258,7 +270,7 @@ extern "C" int relbias_device_status(int reset) {
     return static_cast<int>(v);
 }
 
-extern "C" int relbias_version(void) { return 100; }
+extern "C" int relbias_version(void) { return 200; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"

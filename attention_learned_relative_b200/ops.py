@@ -31,12 +31,12 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 _SZ = ctypes.c_size_t
 SIGNATURES = {
-    "relbias_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
+    "relbias_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "relbias_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
-    "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ,
-                                 _VP]),
+    "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP,
+                                 _SZ, _VP]),
     "relbias_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
-                                         _VP]),
+                                         _I, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_version": (_I, []),
@@ -96,10 +96,12 @@ def _need(cond: bool, msg: str):
 
 
 def attn_fwd(q, k, v, r, w, window: int, R: int, scale: float | None = None, out=None, lse=None,
-             stream=None):
+             stream=None, temp_n0: int = 0):
     """Prefill.  q [B,T,Hq,d], k/v [B,T,Hkv,d] (bf16 or fp32, CUDA, contiguous),
     r [B,T,Hq] fp32, w [Hq,R] fp32.  Returns o [B,T,Hq,d] (and fills `lse`
-    [B,Hq,T] fp32 when given).  scale defaults to 1/sqrt(d)."""
+    [B,Hq,T] fp32 when given).  scale defaults to 1/sqrt(d).  temp_n0 > 1 applies
+    the context-length temperature max(1, ln n / ln temp_n0) to the logits of a row
+    that sees n keys (see include/relbias_attn.h)."""
     _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -116,8 +118,8 @@ def attn_fwd(q, k, v, r, w, window: int, R: int, scale: float | None = None, out
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     rc = lib().relbias_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
-                                B, T, Hq, Hkv, d, int(window), int(R), float(scale), _dtype_code(q),
-                                _stream_handle(stream, q.device))
+                                B, T, Hq, Hkv, d, int(window), int(R), float(scale), int(temp_n0),
+                                _dtype_code(q), _stream_handle(stream, q.device))
     _check(rc)
     return out
 
@@ -128,11 +130,12 @@ def decode_workspace_size(B: int, Hq: int, Hkv: int, n_ctx: int, d: int, window:
 
 
 def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | None = None, out=None,
-                lse=None, workspace=None, stream=None):
+                lse=None, workspace=None, stream=None, temp_n0: int = 0):
     """Decode one query per sequence at position n_ctx-1.  q [B,Hq,d] bf16,
     k_cache/v_cache [B,n_ctx,Hkv,d] bf16, r [B,Hq] fp32, w [Hq,R] fp32.
     Returns o [B,Hq,d] bf16 (fills `lse` [B,Hq] when given).  `workspace` is a
-    byte tensor of at least decode_workspace_size(...) bytes; allocated if None."""
+    byte tensor of at least decode_workspace_size(...) bytes; allocated if None.
+    temp_n0: context-length temperature break point, as for attn_fwd."""
     _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "q [B,Hq,d], cache [B,N,Hkv,d]")
     B, Hq, d = q.shape
     _, N, Hkv, _ = k_cache.shape
@@ -152,14 +155,14 @@ def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | N
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     rc = lib().relbias_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
-                                   B, N, Hq, Hkv, d, int(window), int(R), float(scale), _dtype_code(q),
-                                   _ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
+                                   B, N, Hq, Hkv, d, int(window), int(R), float(scale), int(temp_n0),
+                                   _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
     _check(rc)
     return out
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, r, w, window: int, R: int, scale: float | None = None, out=None,
-                        lse=None, stream=None):
+                        lse=None, stream=None, temp_n0: int = 0):
     """attn_decode for callers that cannot allocate device memory: the split
     partials go to the library's own static scratch (see
     relbias_attn_decode_noalloc in include/relbias_attn.h for its size limit and
@@ -176,7 +179,7 @@ def attn_decode_noalloc(q, k_cache, v_cache, r, w, window: int, R: int, scale: f
         scale = 1.0 / math.sqrt(d)
     rc = lib().relbias_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out),
                                            _ptr(lse), B, N, Hq, Hkv, d, int(window), int(R), float(scale),
-                                           _dtype_code(q), _stream_handle(stream, q.device))
+                                           int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
     _check(rc)
     return out
 

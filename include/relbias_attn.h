@@ -84,6 +84,13 @@ typedef enum {
  *
  *   B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0; window <= 0 means full causal;
  *   R >= 0 (R == 0: no bias); scale > 0 and finite.
+ *   temp_n0: context-length temperature of global layers (the essay, "The
+ *   temperature scale is dependent on context length": queries and position bias
+ *   are both scaled by a factor that is flat up to 128k tokens and grows
+ *   logarithmically beyond; the page's formula is garbled).  Reading taken: a
+ *   row that sees n keys (n = i+1, or min(i+1, window)) has its whole logit
+ *   multiplied by max(1, ln n / ln temp_n0).  temp_n0 <= 1 turns it off; the
+ *   page's break point is 131072.  The LSE is that of the scaled logits.
  *   RELBIAS_BF16 needs a B200-class GPU (compute capability 10.0), d in {64, 128}
  *   and R <= 2048; RELBIAS_FP32 takes d in {32, 64, 128, 256} on any GPU.
  *   The output buffers must not overlap the inputs.
@@ -92,7 +99,7 @@ RELBIAS_API int relbias_attn_fwd(const void* q, const void* k, const void* v,
                      const float* r, const float* w,
                      void* o, float* lse,
                      int B, int T, int Hq, int Hkv, int d,
-                     int window, int R, float scale,
+                     int window, int R, float scale, int temp_n0,
                      int dtype, void* stream);
 
 /*
@@ -114,7 +121,8 @@ RELBIAS_API int relbias_attn_fwd(const void* q, const void* k, const void* v,
  *            contents on entry do not matter and are overwritten.
  *
  *   dtype must be RELBIAS_BF16; d == 128; Hq/Hkv <= 8; n_ctx >= 1; other
- *   argument rules as for relbias_attn_fwd.
+ *   argument rules as for relbias_attn_fwd (the query sees n = n_ctx keys, or
+ *   min(n_ctx, window), for the temperature).
  */
 RELBIAS_API size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d,
                                           int window);
@@ -123,7 +131,7 @@ RELBIAS_API int relbias_attn_decode(const void* q, const void* k_cache, const vo
                         const float* r, const float* w,
                         void* o, float* lse,
                         int B, int n_ctx, int Hq, int Hkv, int d,
-                        int window, int R, float scale,
+                        int window, int R, float scale, int temp_n0,
                         int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /*
@@ -152,7 +160,7 @@ RELBIAS_API int relbias_attn_decode_noalloc(const void* q, const void* k_cache, 
                         const float* r, const float* w,
                         void* o, float* lse,
                         int B, int n_ctx, int Hq, int Hkv, int d,
-                        int window, int R, float scale,
+                        int window, int R, float scale, int temp_n0,
                         int dtype, void* stream);
 
 /* Description of the last failed call on this thread ("" if none).  The string

@@ -38,8 +38,17 @@ def test_every_declared_symbol_is_exported(lib):
         assert name in ops.SIGNATURES, "binding lacks " + name
 
 
+def test_binding_argument_counts_match_header():
+    """Every declaration's parameter count equals the binding's argtypes (catches ABI drift)."""
+    text = open(HEADER).read()
+    for m in re.finditer(r"^RELBIAS_API\s+[\w\s\*]*?\b(\w+)\s*\(([^)]*)\)", text, flags=re.M):
+        name, params = m.group(1), m.group(2).strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(ops.SIGNATURES[name][1]) == n, (name, n, len(ops.SIGNATURES[name][1]))
+
+
 def test_version(lib):
-    assert ops.version() >= 100
+    assert ops.version() >= 200
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
@@ -47,10 +56,11 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails it
 
 def _fwd(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=1, T=8, Hq=4, Hkv=2, d=128,
-             window=0, R=16, scale=0.125, dtype=ops.RELBIAS_BF16)
+             window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_BF16)
     a.update(kw)
     return lib.relbias_attn_fwd(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"], a["T"],
-                                a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["dtype"], None)
+                                a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["temp_n0"],
+                                a["dtype"], None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -92,11 +102,11 @@ def test_r0_needs_no_table(lib):
 
 def _dec(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=2, N=100, Hq=8, Hkv=1, d=128,
-             window=0, R=16, scale=0.1, dtype=ops.RELBIAS_BF16, ws=FAKE, ws_bytes=1 << 20)
+             window=0, R=16, scale=0.1, temp_n0=0, dtype=ops.RELBIAS_BF16, ws=FAKE, ws_bytes=1 << 20)
     a.update(kw)
     return lib.relbias_attn_decode(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"], a["N"],
-                                   a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["dtype"],
-                                   a["ws"], a["ws_bytes"], None)
+                                   a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"], a["temp_n0"],
+                                   a["dtype"], a["ws"], a["ws_bytes"], None)
 
 
 @pytest.mark.parametrize("kw,code", [

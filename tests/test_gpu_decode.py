@@ -45,6 +45,20 @@ def _run(x, window, R, scale):
     return o, lse
 
 
+@pytest.mark.parametrize("B,N,Hq,Hkv,window,R,n0", [
+    (2, 3000, 8, 2, 0, 512, 1000),     # tau = ln 3000 / ln 1000
+    (1, 5000, 16, 4, 512, 512, 100),   # windowed: the query sees 512 keys
+])
+def test_decode_context_length_temperature(B, N, Hq, Hkv, window, R, n0):
+    x = _inputs(B, N, Hq, Hkv, 128, R, seed=N + n0)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device="cuda")
+    o = ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], window, R, 0.0884, lse=lse, temp_n0=n0)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = O.attn_decode(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), window, R,
+                                   0.0884, temp_n0=n0)
+    assert_bf16_close(o, o_ref, lse, lse_ref, "decode temperature %s" % ((B, N, Hq, Hkv, window, R, n0),))
+
+
 DECODE_CASES = [
     # B, N,     Hq, Hkv, window, R
     (2, 1, 8, 1, 0, 16),          # cache holds only the query's own row

@@ -110,6 +110,37 @@ def test_bf16_other_scale_and_large_logits():
         assert_bf16_close(o, o_ref, lse, lse_ref, "scale %g" % scale)
 
 
+@pytest.mark.parametrize("dtype,B,T,Hq,Hkv,d,window,R,n0", [
+    (torch.bfloat16, 1, 700, 8, 2, 128, 0, 256, 200),      # global layer: rows past 200 keys are sharpened
+    (torch.bfloat16, 1, 900, 4, 2, 128, 512, 512, 300),    # windowed: n saturates at the window
+    (torch.bfloat16, 1, 400, 8, 1, 64, 0, 64, 50),
+    (torch.float32, 1, 300, 4, 2, 64, 0, 64, 40),
+    (torch.float32, 1, 300, 4, 2, 128, 100, 30, 20),
+])
+def test_context_length_temperature(dtype, B, T, Hq, Hkv, d, window, R, n0):
+    """Logits of a row that sees n > n0 keys scaled by ln n / ln n0 (content and bias)."""
+    x = _inputs(B, T, Hq, Hkv, d, R, seed=T + n0, dtype=dtype)
+    scale = 1.0 / math.sqrt(d)
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], window, R, scale, lse=lse, temp_n0=n0)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), window,
+                                    R, scale, temp_n0=n0)
+    check = assert_fp32_close if dtype == torch.float32 else assert_bf16_close
+    check(o, o_ref, lse, lse_ref, "temperature %s" % ((dtype, B, T, Hq, Hkv, d, window, R, n0),))
+
+
+def test_temperature_off_is_bitwise_identical():
+    """A break point that no row's key count exceeds leaves every output bit unchanged."""
+    x = _inputs(1, 500, 8, 2, 128, 128, seed=41)
+    o0, l0 = _run(x, 0, 128, 0.09)
+    for n0 in (1, 500, 100000):
+        lse = torch.empty_like(l0)
+        o1 = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], 0, 128, 0.09, lse=lse, temp_n0=n0)
+        torch.cuda.synchronize()
+        assert torch.equal(o0, o1) and torch.equal(l0, lse)
+
+
 def test_deterministic():
     x = _inputs(1, 1000, 8, 2, 128, 512, seed=3)
     o1, l1 = _run(x, 512, 512, 0.088)

@@ -41,7 +41,7 @@ def _noalloc_call(lib, x, window, R, scale, o, lse):
     _, N, Hkv, _ = x["k"].shape
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return lib.relbias_attn_decode_noalloc(_p(x["q"]), _p(x["k"]), _p(x["v"]), _p(x["r"]), _p(x["w"]), _p(o),
-                                           _p(lse), B, N, Hq, Hkv, d, window, R, scale, ops.RELBIAS_BF16, stream)
+                                           _p(lse), B, N, Hq, Hkv, d, window, R, scale, 0, ops.RELBIAS_BF16, stream)
 
 
 def test_noalloc_decode_matches_regular_entry_point_twice():
@@ -82,6 +82,6 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     lse = torch.empty(B, Hq, device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     rc = lib.relbias_attn_decode_noalloc(_p(x["q"]), _p(x["k"]), _p(x["v"]), _p(x["r"]), _p(x["w"]), _p(o),
-                                         _p(lse), B, N, Hq, Hkv, d, 0, R, 0.1, ops.RELBIAS_BF16, stream)
+                                         _p(lse), B, N, Hq, Hkv, d, 0, R, 0.1, 0, ops.RELBIAS_BF16, stream)
     assert rc == ops.RELBIAS_ERR_UNSUPPORTED
     assert "static scratch" in ops.last_error()
