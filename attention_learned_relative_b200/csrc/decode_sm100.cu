@@ -16,6 +16,15 @@
 // warps take chunks round-robin and merge their running (max, sum, output) in
 // shared memory; each CTA writes one partial per query head to the workspace.  The
 // combine kernel merges the partials of a (b, h) with one warp.
+//
+// Paged, variable-length caches (PAGED = true): keys live in a pool of pages of
+// page_size rows (a multiple of the 32-key chunk), sequence b's logical block k in
+// page block_table[b][k], and each sequence has its own length seq_lens[b] -- the
+// paged KV cache and variable sequence lengths the essay's kernel-cost section lists
+// among what a production attention kernel covers.  Chunks then start at multiples
+// of 32 (so each lies in one page), keys before a window's start are masked, and a
+// split that lies past a short sequence's end writes an empty partial (max -inf),
+// which the combine skips.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -86,6 +95,7 @@ __device__ __forceinline__ uint32_t swz(int key, int dcol) {
     return box * kBoxBytes + key * 128 + ((ch ^ (key & 7)) << 4);
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kDThreads, 1)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const DecodeParams p) {
@@ -96,9 +106,25 @@ __global__ void __launch_bounds__(kDThreads, 1)
 
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // This sequence's length, first attended row, chunk grid and logit scale.
+    int N = p.N, key_lo = p.key_lo, chunk0 = p.key_lo, nchunks = p.nchunks;
+    float c1 = p.scale_log2;
+    if constexpr (PAGED) {
+        N = p.seq_lens[b];
+        if (N < 1 || N > p.N) {
+            // Outside [1, max_seq_len]: clamp (block-table reads stay in bounds) and report.
+            if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadLength);
+            N = min(max(N, 1), p.N);
+        }
+        key_lo = p.window > 0 ? max(0, N - p.window) : 0;
+        chunk0 = (key_lo / kChunk) * kChunk;
+        nchunks = (N - chunk0 + kChunk - 1) / kChunk;
+        const int nk = N - key_lo;   // keys the query sees, for the temperature
+        if (p.temp_n0 > 1 && nk > p.temp_n0) c1 *= __logf(static_cast<float>(nk)) * p.inv_log_n0;
+    }
     const int c_begin = split * p.chunks_per_split;
-    const int c_end = min(p.nchunks, c_begin + p.chunks_per_split);
-    const int nloc = c_end - c_begin;
+    const int c_end = min(nchunks, c_begin + p.chunks_per_split);
+    const int nloc = max(0, c_end - c_begin);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDStages; ++s) {
@@ -119,13 +145,21 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 const int st = li % kDStages;
                 const uint32_t ph = (li / kDStages) & 1;
                 if (!mbar_wait(&bars->empty[st], ph ^ 1, abort_flag)) break;
-                const int key0 = p.key_lo + (c_begin + li) * kChunk;
+                const int key0 = chunk0 + (c_begin + li) * kChunk;
+                int row = key0, seq = b;   // token and sequence coordinates of the chunk
+                if constexpr (PAGED) {
+                    // key0 < N <= max_pages * page_size, so the table read is in bounds; a
+                    // page index outside the pool reads zeros (TMA fills out-of-range rows).
+                    seq = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + key0 / p.page_size);
+                    row = key0 % p.page_size;
+                    if (seq < 0 || seq >= p.num_pages) atomicOr(&g_status, kStatusBadLength);
+                }
                 mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
                 uint8_t* base = sm->stages[st];
-                tma_load_4d(base, &tm_k, &bars->full[st], 0, g, key0, b);
-                tma_load_4d(base + kBoxBytes, &tm_k, &bars->full[st], 64, g, key0, b);
-                tma_load_4d(base + 2 * kBoxBytes, &tm_v, &bars->full[st], 0, g, key0, b);
-                tma_load_4d(base + 3 * kBoxBytes, &tm_v, &bars->full[st], 64, g, key0, b);
+                tma_load_4d(base, &tm_k, &bars->full[st], 0, g, row, seq);
+                tma_load_4d(base + kBoxBytes, &tm_k, &bars->full[st], 64, g, row, seq);
+                tma_load_4d(base + 2 * kBoxBytes, &tm_v, &bars->full[st], 0, g, row, seq);
+                tma_load_4d(base + 3 * kBoxBytes, &tm_v, &bars->full[st], 64, g, row, seq);
             }
             // Do not leave while copies into this CTA's shared memory are in flight.
             int dummy = 0;
@@ -138,7 +172,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // -------------------------------------------------------------------- consumers
     const int gq = lane >> 2;        // fragment row group
     const int qq = lane & 3;         // fragment column pair
-    const float c1 = p.scale_log2;
 
     // q^T as B fragments (head dim = K, heads of the group = N), padded with zero heads.
     uint32_t qb[kD / 16][2];
@@ -170,7 +203,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
     for (int dt = 0; dt < kD / 16; ++dt) oacc[dt][0] = oacc[dt][1] = oacc[dt][2] = oacc[dt][3] = 0.0f;
 
-    const int last = p.N - 1;
+    const int last = N - 1;
     bool ok = true;
     for (int li = warp; li < nloc; li += kConsumers) {
         const int st = li % kDStages;
@@ -179,7 +212,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         if (!ok) break;
         const uint32_t kbase = smem_u32(sm->stages[st]);
         const uint32_t vbase = kbase + 2 * kBoxBytes;
-        const int key0 = p.key_lo + (c_begin + li) * kChunk;
+        const int key0 = chunk0 + (c_begin + li) * kChunk;
 
         // S^T = K q^T for the chunk's groups of 16 keys.
         float sacc[kMT][4];
@@ -197,7 +230,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         }
 
         // Logits in log2 units, bias on the last R rows, mask rows past the cache end.
-        const bool biased = key0 + kChunk - 1 >= p.N - p.R;
+        const bool biased = key0 + kChunk - 1 >= N - p.R;
         float mc[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int mt = 0; mt < kMT; ++mt) {
@@ -211,7 +244,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
                     if (dist >= 0 && dist < p.R)
                         x = fmaf(rs[col], __ldg(p.w + static_cast<size_t>(hcol[col]) * p.R + dist), x);
                 }
-                x = (key <= last) ? x * c1 : -INFINITY;
+                bool visible = key <= last;
+                if constexpr (PAGED) visible = visible && key >= key_lo;   // aligned chunks start early
+                x = visible ? x * c1 : -INFINITY;
                 sacc[mt][e] = x;
                 mc[col] = fmaxf(mc[col], x);
             }
@@ -235,6 +270,22 @@ __global__ void __launch_bounds__(kDThreads, 1)
             }
             m_run[col] = m_new;
             base[col] = (m_new == -INFINITY) ? 0.0f : m_new;
+        }
+        if constexpr (PAGED) {
+            // Rows past the sequence's end in its last page hold whatever the pool had
+            // there; their P is 0, but 0 * NaN is not, so zero those V rows first.  A row
+            // of a 64-column box is 128 contiguous bytes (the swizzle permutes chunks
+            // within it).
+            const int first_dead = last - key0 + 1;
+            if (first_dead < kChunk) {
+                const int nb = (kChunk - first_dead) * 2 * 8;   // rows x boxes x 16-byte chunks
+                for (int x = lane; x < nb; x += 32) {
+                    const int rr = first_dead + x / 16, box = (x >> 3) & 1, ch = x & 7;
+                    *reinterpret_cast<uint4*>(sm->stages[st] + 2 * kBoxBytes + box * kBoxBytes + rr * 128 + ch * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
         }
         // P^T (keys x heads) -> bf16 -> transposed 8x8 blocks = B fragments.
         uint32_t pb[kMT][2];
@@ -370,17 +421,30 @@ size_t decode_workspace_bytes(int B, int Hq, int nsplit, int d) {
     return static_cast<size_t>(B) * Hq * nsplit * (d + 4) * sizeof(float);
 }
 
-cudaError_t launch_decode_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
-                               cudaStream_t stream) {
+namespace {
+template <bool PAGED>
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
     const int smem = static_cast<int>(sizeof(DecodeSmem)) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_splitkv_kernel<PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.nsplit, p.Hkv, p.B);
-    decode_splitkv_kernel<<<grid, kDThreads, smem, stream>>>(tk, tv, p);
+    decode_splitkv_kernel<PAGED><<<grid, kDThreads, smem, stream>>>(tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine_kernel<<<(p.B * p.Hq + 3) / 4, 128, 0, stream>>>(p);
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_decode_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                               cudaStream_t stream) {
+    return launch_decode<false>(tk, tv, p, stream);
+}
+
+cudaError_t launch_decode_paged_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                                     cudaStream_t stream) {
+    return launch_decode<true>(tk, tv, p, stream);
 }
 
 }  // namespace relbias

@@ -55,10 +55,22 @@ struct DecodeParams {
     int chunks_per_split;
     float scale_log2;
     float inv_scale;
+    // Paged, variable-length caches (decode_splitkv_kernel<true>): the cache is a pool
+    // of pages [num_pages, page_size, Hkv, d]; sequence b's logical block k lives in
+    // page block_table[b * max_pages + k]; its length is seq_lens[b] (<= N, the bound
+    // the splits are planned for).  key_lo / nchunks are then per sequence.
+    const int* block_table;
+    const int* seq_lens;
+    int page_size, max_pages, num_pages;
+    int temp_n0;             // > 1: per-sequence context-length temperature
+    float inv_log_n0;
 };
 int decode_num_splits(int B, int Hkv, int N, int window, int num_sms);
 size_t decode_workspace_bytes(int B, int Hq, int nsplit, int d);
 cudaError_t launch_decode_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                                cudaStream_t stream);
+// tk/tv: tensor maps over the page pool (make_map with B = num_pages, T = page_size).
+cudaError_t launch_decode_paged_bf16(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                                     cudaStream_t stream);
 
 }  // namespace relbias

@@ -12,6 +12,7 @@ namespace relbias {
 __device__ unsigned int g_status = 0;
 
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusBadLength = 2u;   // a device-side length or page index was out of range
 constexpr float kLn2 = 0.6931471805599453f;
 // A single wait longer than this is treated as a hang (nanoseconds).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -253,6 +253,105 @@ extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const voi
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "decode launch");
 }
 
+namespace relbias {
+namespace {
+// Split plan for paged decode: the longest chunk run any sequence of at most
+// max_seq_len rows can need (chunks aligned to multiples of 32 rows).
+int paged_max_chunks(int max_seq_len, int window) {
+    const int all = (max_seq_len + kChunk - 1) / kChunk;
+    if (window <= 0) return all;
+    return std::min(all, (window + kChunk - 1) / kChunk + 1);
+}
+int paged_num_splits(int B, int Hkv, int max_chunks, int num_sms) {
+    const int target = num_sms * 8;
+    const int pairs = std::max(1, B * Hkv);
+    int nsplit = std::max(1, std::min((target + pairs - 1) / pairs, max_chunks));
+    const int cps = (max_chunks + nsplit - 1) / nsplit;
+    return (max_chunks + cps - 1) / cps;
+}
+}  // namespace
+}  // namespace relbias
+
+extern "C" size_t relbias_attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_seq_len, int d,
+                                                          int window) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_seq_len < 1 || d < 1) return 0;
+    DeviceInfo dev;
+    if (device_info(dev) != RELBIAS_OK) return 0;
+    const int nsplit = paged_num_splits(B, Hkv, paged_max_chunks(max_seq_len, window > 0 ? window : 0), dev.sms);
+    return decode_workspace_bytes(B, Hq, nsplit, d);
+}
+
+extern "C" int relbias_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                         const int* block_table, const int* seq_lens, const float* r, const float* w,
+                                         void* o, float* lse, int B, int num_pages, int page_size, int max_pages,
+                                         int max_seq_len, int Hq, int Hkv, int d, int window, int R, float scale,
+                                         int temp_n0, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+    t_err.clear();
+    int rc = check_common(B, max_seq_len, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0) return RELBIAS_OK;
+    if (max_seq_len < 1) return fail(RELBIAS_ERR_ARG, "max_seq_len (%d) must be >= 1", max_seq_len);
+    if (num_pages < 1 || max_pages < 1)
+        return fail(RELBIAS_ERR_ARG, "num_pages (%d) and max_pages (%d) must be >= 1", num_pages, max_pages);
+    if (page_size < kChunk || page_size % kChunk != 0)
+        return fail(RELBIAS_ERR_ARG, "page_size (%d) must be a positive multiple of %d", page_size, kChunk);
+    if (static_cast<long long>(max_pages) * page_size < max_seq_len)
+        return fail(RELBIAS_ERR_ARG, "max_pages * page_size (%lld) is shorter than max_seq_len (%d)",
+                    static_cast<long long>(max_pages) * page_size, max_seq_len);
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !r || !o || !workspace)
+        return fail(RELBIAS_ERR_ARG, "q, k_pages, v_pages, block_table, seq_lens, r, o and workspace must not be null");
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
+        return fail(RELBIAS_ERR_ARG, "q, k_pages, v_pages, o and workspace must be 16-byte aligned");
+    if (!aligned4(r) || !aligned4(block_table) || !aligned4(seq_lens) || (lse && !aligned4(lse)))
+        return fail(RELBIAS_ERR_ARG, "r, block_table, seq_lens and lse must be 4-byte aligned");
+    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports bf16 only");
+    if (d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports d == 128, got %d", d);
+    if (Hq / Hkv > 8) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports up to 8 query heads per key/value head");
+    DeviceInfo dev;
+    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "decode needs compute capability 10.0 (sm_100a), found %d.%d", dev.major,
+                    dev.minor);
+
+    DecodeParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.r = r;
+    p.w = w;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.part = static_cast<float*>(workspace);
+    p.B = B;
+    p.N = max_seq_len;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.window = window > 0 ? window : 0;
+    p.R = R;
+    p.key_lo = 0;
+    p.nchunks = paged_max_chunks(max_seq_len, p.window);
+    p.nsplit = paged_num_splits(B, Hkv, p.nchunks, dev.sms);
+    p.chunks_per_split = (p.nchunks + p.nsplit - 1) / p.nsplit;
+    p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.page_size = page_size;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.temp_n0 = temp_n0 > 1 ? temp_n0 : 0;
+    p.inv_log_n0 = temp_n0 > 1 ? static_cast<float>(1.0 / std::log(static_cast<double>(temp_n0))) : 0.0f;
+    const size_t need = decode_workspace_bytes(B, Hq, p.nsplit, d);
+    if (ws_bytes < need)
+        return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes, need);
+
+    CUtensorMap tk, tv;
+    if ((rc = make_map(&tk, k_pages, num_pages, page_size, Hkv, d, kChunk)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v_pages, num_pages, page_size, Hkv, d, kChunk)) != RELBIAS_OK) return rc;
+    cudaError_t e = launch_decode_paged_bf16(tk, tv, p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "paged decode launch");
+}
+
 extern "C" const char* relbias_last_error(void) { return t_err.c_str(); }
 
 extern "C" int relbias_device_status(int reset) {

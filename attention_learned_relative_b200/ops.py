@@ -22,6 +22,7 @@ RELBIAS_ERR_ARG = -1
 RELBIAS_ERR_UNSUPPORTED = -2
 RELBIAS_ERR_CUDA = -3
 RELBIAS_STATUS_TIMEOUT = 1
+RELBIAS_STATUS_BAD_LENGTH = 2
 RELBIAS_BF16 = 0
 RELBIAS_FP32 = 1
 
@@ -37,6 +38,9 @@ SIGNATURES = {
                                  _SZ, _VP]),
     "relbias_attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                          _I, _VP]),
+    "relbias_attn_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "relbias_attn_decode_paged": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
+                                       _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_version": (_I, []),
@@ -180,6 +184,50 @@ def attn_decode_noalloc(q, k_cache, v_cache, r, w, window: int, R: int, scale: f
     rc = lib().relbias_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(r), _ptr(w), _ptr(out),
                                            _ptr(lse), B, N, Hq, Hkv, d, int(window), int(R), float(scale),
                                            int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def decode_paged_workspace_size(B: int, Hq: int, Hkv: int, max_seq_len: int, d: int, window: int) -> int:
+    """Bytes of device scratch relbias_attn_decode_paged needs for this shape."""
+    return int(lib().relbias_attn_decode_paged_workspace_size(B, Hq, Hkv, max_seq_len, d, int(window)))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, r, w, window: int, R: int, max_seq_len: int,
+                      scale: float | None = None, out=None, lse=None, workspace=None, stream=None,
+                      temp_n0: int = 0):
+    """Decode against a paged, variable-length cache.  q [B,Hq,d] bf16,
+    k_pages/v_pages [num_pages,page_size,Hkv,d] bf16, block_table [B,max_pages] int32,
+    seq_lens [B] int32 (each in [1, max_seq_len]), r [B,Hq] fp32, w [Hq,R] fp32.
+    Sequence b's query sits at position seq_lens[b]-1; its cache row t is row
+    t % page_size of page block_table[b, t // page_size].  Returns o [B,Hq,d]."""
+    _need(q.dim() == 3 and k_pages.dim() == 4 and v_pages.shape == k_pages.shape,
+          "q [B,Hq,d], pages [num_pages,page_size,Hkv,d]")
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_pages.shape
+    _need(dk == d, "page head dim %d != q head dim %d" % (dk, d))
+    _need(q.dtype == k_pages.dtype == v_pages.dtype, "q and pages must share a dtype")
+    _need(block_table.dim() == 2 and block_table.shape[0] == B and block_table.dtype == torch.int32,
+          "block_table must be int32 [B, max_pages]")
+    _need(seq_lens.shape == (B,) and seq_lens.dtype == torch.int32, "seq_lens must be int32 [B]")
+    _need(r.shape == (B, Hq) and r.dtype == torch.float32, "r must be fp32 [B,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    for t in (q, k_pages, v_pages, block_table, seq_lens, r, w, out, lse, workspace):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(lse is None or (lse.shape == (B, Hq) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq]")
+    need = decode_paged_workspace_size(B, Hq, Hkv, max_seq_len, d, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                                         _ptr(r), _ptr(w), _ptr(out), _ptr(lse), B, num_pages, page_size,
+                                         block_table.shape[1], int(max_seq_len), Hq, Hkv, d, int(window), int(R),
+                                         float(scale), int(temp_n0), _dtype_code(q), _ptr(workspace), ws_bytes,
+                                         _stream_handle(stream, q.device))
     _check(rc)
     return out
 

@@ -33,6 +33,7 @@ class Workload:
     dtype: str        # "fp32" or "bf16"
     decode: bool = False
     qk_std: float = 1.0   # Q and K are drawn as N(0, qk_std^2)
+    page_size: int = 0    # decode only: > 0 stores the cache as shuffled pages of this many rows
 
     @property
     def scale(self) -> float:
@@ -77,6 +78,10 @@ WORKLOADS = {
                  R=1024, seed=3, dtype="bf16", qk_std=0.5),
         Workload("global_decode_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0, R=1024,
                  seed=4, dtype="bf16", decode=True),
+        # The same decode step against a paged cache: 256-row pages in a pool whose
+        # block table is a seeded random permutation (scattered physical pages).
+        Workload("global_decode_paged_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0,
+                 R=1024, seed=4, dtype="bf16", decode=True, page_size=256),
     ]
 }
 
@@ -86,6 +91,11 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
 
     Prefill: q [B,T,Hq,d], k/v [B,T,Hkv,d] (wl dtype), r [B,T,Hq] fp32, w [Hq,R] fp32.
     Decode:  q [B,Hq,d], k/v [B,T,Hkv,d] (the cache), r [B,Hq] fp32, w [Hq,R] fp32.
+    Paged decode (page_size > 0) adds k_pages/v_pages [B*T/page_size, page_size, Hkv, d]
+    (the same storage as k/v, read as a page pool), table [B, T/page_size] int32 (a
+    seeded permutation of the pool: sequence b's logical block j is page table[b, j])
+    and lens [B] int32.  The logical cache of sequence b is then k_pages[table[b]],
+    not k[b]; logical_cache() returns it.
     """
     T = wl.T if T is None else T
     B = wl.B if B is None else B
@@ -100,4 +110,28 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
     k = synth.normal((B, T, wl.Hkv, wl.d), s, "k", std=wl.qk_std, dtype=dt, device=device)
     v = synth.normal((B, T, wl.Hkv, wl.d), s, "v", dtype=dt, device=device)
     w = synth.normal((wl.Hq, wl.R), s, "w", std=0.5, device=device)
-    return {"q": q, "k": k, "v": v, "r": r, "w": w}
+    x = {"q": q, "k": k, "v": v, "r": r, "w": w}
+    if wl.decode and wl.page_size > 0:
+        if T % wl.page_size != 0:
+            raise ValueError("paged workload needs T (%d) divisible by page_size (%d)" % (T, wl.page_size))
+        npb = T // wl.page_size
+        x["k_pages"] = k.view(B * npb, wl.page_size, wl.Hkv, wl.d)
+        x["v_pages"] = v.view(B * npb, wl.page_size, wl.Hkv, wl.d)
+        g = torch.Generator().manual_seed(s + 77)
+        x["table"] = torch.randperm(B * npb, generator=g).to(torch.int32).reshape(B, npb).to(device)
+        x["lens"] = torch.full((B,), T, dtype=torch.int32, device=device)
+    return x
+
+
+def logical_cache(x, b: int, kv: int | None = None):
+    """(K, V) of sequence b in logical row order, [T, Hkv, d] (or [T, 1, d] for one
+    key/value head), gathered through the block table for a paged workload."""
+    if "table" not in x:
+        ks, vs = x["k"][b], x["v"][b]
+    else:
+        pages = x["table"][b].long()
+        ks = x["k_pages"][pages].flatten(0, 1)
+        vs = x["v_pages"][pages].flatten(0, 1)
+    if kv is not None:
+        ks, vs = ks[:, kv:kv + 1], vs[:, kv:kv + 1]
+    return ks, vs

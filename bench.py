@@ -193,7 +193,12 @@ def make_sets(wl, nsets, device):
 
 
 def step_fn(wl, ops, workspace):
-    if wl.decode:
+    if wl.decode and wl.page_size > 0:
+        def step(x, stream):
+            ops.attn_decode_paged(x["q"], x["k_pages"], x["v_pages"], x["table"], x["lens"], x["r"], x["w"],
+                                  wl.window, wl.R, wl.T, wl.scale, out=x["o"], lse=x["lse"], workspace=workspace,
+                                  stream=stream)
+    elif wl.decode:
         def step(x, stream):
             ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
                             lse=x["lse"], workspace=workspace, stream=stream)
@@ -211,6 +216,7 @@ def cpu_baseline(wl, x, budget_s):
     import numpy as np
     import torch
     from oracle import oracle as O
+    from attention_learned_relative_b200.workloads import logical_cache
 
     g = torch.Generator().manual_seed(12345)
     if wl.decode:
@@ -222,8 +228,8 @@ def cpu_baseline(wl, x, budget_s):
             b = int(torch.randint(0, wl.B, (1,), generator=g))
             kv = int(torch.randint(0, wl.Hkv, (1,), generator=g))
             heads = list(range(kv * G, (kv + 1) * G))
-            k_sl = x["k"][b:b + 1, :, kv:kv + 1, :].cpu()
-            v_sl = x["v"][b:b + 1, :, kv:kv + 1, :].cpu()
+            k_sl, v_sl = logical_cache(x, b, kv)
+            k_sl, v_sl = k_sl[None].cpu(), v_sl[None].cpu()
             q = x["q"][b, heads].float().cpu()
             r = x["r"][b, heads].cpu().reshape(G, 1)
             proj = x["w"][heads].cpu().reshape(G, 1, wl.R)
@@ -297,7 +303,10 @@ def run_ours(args, wl, peaks, peaks_kind):
     sets = make_sets(wl, nsets, dev)
     workspace = None
     if wl.decode:
-        nbytes = ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
+        if wl.page_size > 0:
+            nbytes = ops.decode_paged_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
+        else:
+            nbytes = ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     step = step_fn(wl, ops, workspace)
     stream = torch.cuda.current_stream(dev)
@@ -404,6 +413,7 @@ def run_ours(args, wl, peaks, peaks_kind):
             "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
                        "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
+                       **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
                        "parallelism": "dp%d (batch shards, no collective)" % world,
                        "l2": ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6))
                        if nsets > 1 else "per-step input %.0f MB > L2" % (step_bytes / 1e6)},

@@ -63,6 +63,7 @@ extern "C" {
 
 /* Bits of the device-side status word (relbias_device_status). */
 #define RELBIAS_STATUS_TIMEOUT   1u /* a bounded wait inside a kernel ran out             */
+#define RELBIAS_STATUS_BAD_LENGTH 2u /* a device-side sequence length or page index was out of range */
 
 /* Element type of q, k, v and o.  r, w and lse are always fp32. */
 typedef enum {
@@ -162,6 +163,40 @@ RELBIAS_API int relbias_attn_decode_noalloc(const void* q, const void* k_cache, 
                         int B, int n_ctx, int Hq, int Hkv, int d,
                         int window, int R, float scale, int temp_n0,
                         int dtype, void* stream);
+
+/*
+ * Decode against a paged, variable-length KV cache: the "paged KV, variable seq
+ * len" a production attention kernel must cover (the essay "Thinking Machines
+ * dropped RoPE", closing section on kernel cost).  Same computation as
+ * relbias_attn_decode for each sequence b, whose query sits at position
+ * seq_lens[b]-1 and whose cache rows live in pages:
+ *
+ *   k_pages, v_pages [num_pages, page_size, Hkv, d]  bf16   the page pool
+ *   block_table      [B, max_pages]                 int32  page of each logical
+ *                    block of page_size rows (row t of sequence b is row
+ *                    t % page_size of page block_table[b][t / page_size])
+ *   seq_lens         [B]                            int32  rows of each sequence
+ *                    (device memory, read by the kernel; 1 <= seq_lens[b] <= max_seq_len)
+ *   q [B, Hq, d], r [B, Hq], w [Hq, R], o [B, Hq, d], lse [B, Hq]: as for decode.
+ *
+ *   page_size: a positive multiple of 32.  max_pages * page_size >= max_seq_len.
+ *   max_seq_len bounds every seq_lens[b] and plans the key splits;
+ *   workspace: at least relbias_attn_decode_paged_workspace_size(...) bytes.
+ *   A length outside [1, max_seq_len] is clamped into it, and a page index outside
+ *   the pool reads zeros; either sets RELBIAS_STATUS_BAD_LENGTH in the device
+ *   status word (relbias_device_status).  Other rules as for relbias_attn_decode.
+ */
+RELBIAS_API size_t relbias_attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_seq_len, int d,
+                                                int window);
+
+RELBIAS_API int relbias_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                        const int* block_table, const int* seq_lens,
+                        const float* r, const float* w,
+                        void* o, float* lse,
+                        int B, int num_pages, int page_size, int max_pages, int max_seq_len,
+                        int Hq, int Hkv, int d,
+                        int window, int R, float scale, int temp_n0,
+                        int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* Description of the last failed call on this thread ("" if none).  The string
  * stays valid until the next library call on the same thread. */

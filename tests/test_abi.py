@@ -131,3 +131,34 @@ def test_decode_empty_batch(lib):
 def test_workspace_size_rejects_bad_shapes(lib):
     assert ops.decode_workspace_size(0, 8, 1, 100, 128, 0) == 0
     assert ops.decode_workspace_size(1, 8, 3, 100, 128, 0) == 0
+
+
+def _paged(lib, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=2, num_pages=10,
+             page_size=64, max_pages=5, max_seq_len=300, Hq=8, Hkv=2, d=128, window=0, R=16, scale=0.1, temp_n0=0,
+             dtype=ops.RELBIAS_BF16, ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    return lib.relbias_attn_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["sl"], a["r"], a["w"], a["o"],
+                                         a["lse"], a["B"], a["num_pages"], a["page_size"], a["max_pages"],
+                                         a["max_seq_len"], a["Hq"], a["Hkv"], a["d"], a["window"], a["R"],
+                                         a["scale"], a["temp_n0"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(page_size=48), ops.RELBIAS_ERR_ARG),          # not a multiple of 32
+    (dict(page_size=0), ops.RELBIAS_ERR_ARG),
+    (dict(max_pages=4), ops.RELBIAS_ERR_ARG),           # 4 * 64 < max_seq_len 300
+    (dict(num_pages=0), ops.RELBIAS_ERR_ARG),
+    (dict(max_seq_len=0), ops.RELBIAS_ERR_ARG),
+    (dict(bt=None), ops.RELBIAS_ERR_ARG),
+    (dict(sl=None), ops.RELBIAS_ERR_ARG),
+    (dict(sl=FAKE + 2), ops.RELBIAS_ERR_ARG),           # misaligned
+    (dict(Hq=9), ops.RELBIAS_ERR_ARG),
+])
+def test_paged_decode_rejects_bad_arguments(lib, kw, code):
+    assert _paged(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_paged_decode_batch_zero_is_a_no_op(lib):
+    assert _paged(lib, B=0) == ops.RELBIAS_OK
