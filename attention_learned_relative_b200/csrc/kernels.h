@@ -19,6 +19,8 @@ struct PrefillParams {
     int HP;                  // G / nslots: head pairs per key/value head
     int window, R;
     int n_qt;                // ceil(T / 128)
+    int q_off;               // position of query row 0 (a chunk after a cached prefix; 0 otherwise)
+    int kv_T;                // rows of K/V (>= q_off + T)
     int total_items;         // n_qt * B * Hkv * HP
     int o_v8;                // 1: o is 32-byte aligned (rows are written with 32-byte stores)
     int contiguous;          // 1: each CTA takes a contiguous run of items, query tiles innermost
@@ -36,8 +38,8 @@ cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& 
 
 // fp32 SIMT prefill (prefill_fp32.cu).
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
-                                float* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, int temp_n0, cudaStream_t stream);
+                                float* o, float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
+                                int window, int R, float scale, int temp_n0, cudaStream_t stream);
 
 // bf16 split-KV decode + log-sum-exp combine (decode_sm100.cu).
 struct DecodeParams {

@@ -25,8 +25,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreadsF32)
     prefill_fp32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                         const float* __restrict__ r, const float* __restrict__ w, float* __restrict__ o,
-                        float* __restrict__ lse, int T, int Hq, int Hkv, int window, int R, float scale,
-                        int temp_n0) {
+                        float* __restrict__ lse, int T, int q_off, int kv_T, int Hq, int Hkv, int window, int R,
+                        float scale, int temp_n0) {
     constexpr int BK = D <= 128 ? 32 : 16;   // keys per shared-memory tile
     constexpr int DL = D / 4;                 // dims per lane
     __shared__ __align__(16) float ks[BK * D];
@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kThreadsF32)
     const int row = threadIdx.x >> 2, qd = threadIdx.x & 3;
     const int i = i0 + row;
     const bool row_ok = i < T;
+    const int pos = q_off + i;   // the row's position in the sequence (K/V have kv_T rows)
+    const int kv_end = q_off + T;   // keys past the chunk's last row are never visible: never read
 
     float qv[DL], ov[DL];
     const float* qrow = q + ((static_cast<size_t>(b) * T + (row_ok ? i : 0)) * Hq + h) * D;
@@ -50,7 +52,7 @@ __global__ void __launch_bounds__(kThreadsF32)
     // terms scaled by ln n / ln temp_n0.
     float tau = 1.0f;
     if (temp_n0 > 1) {
-        const int n = window > 0 ? min(i + 1, window) : i + 1;
+        const int n = window > 0 ? min(pos + 1, window) : pos + 1;
         if (n > temp_n0) tau = static_cast<float>(log(static_cast<double>(n)) / log(static_cast<double>(temp_n0)));
     }
     const float ri = row_ok ? tau * r[(static_cast<size_t>(b) * T + i) * Hq + h] : 0.0f;
@@ -58,16 +60,16 @@ __global__ void __launch_bounds__(kThreadsF32)
     float m = -INFINITY, l = 0.0f;
 
     int j_begin = 0;
-    if (window > 0) j_begin = max(0, i0 - window + 1);
-    const int j_end = min(T, i0 + kRows);   // exclusive
+    if (window > 0) j_begin = max(0, q_off + i0 - window + 1);
+    const int j_end = min(kv_end, q_off + i0 + kRows);   // exclusive
     for (int j0 = j_begin; j0 < j_end; j0 += BK) {
         __syncthreads();
         for (int x = threadIdx.x; x < BK * D / 4; x += kThreadsF32) {
             const int jj = (4 * x) / D, c = (4 * x) % D;
             const int j = j0 + jj;
             float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), vv = kk;
-            if (j < T) {
-                const size_t off = ((static_cast<size_t>(b) * T + j) * Hkv + g) * D + c;
+            if (j < kv_end) {
+                const size_t off = ((static_cast<size_t>(b) * kv_T + j) * Hkv + g) * D + c;
                 kk = *reinterpret_cast<const float4*>(k + off);
                 vv = *reinterpret_cast<const float4*>(v + off);
             }
@@ -86,8 +88,8 @@ __global__ void __launch_bounds__(kThreadsF32)
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
             const int j = j0 + jj;
-            const int dist = i - j;
-            const bool valid = row_ok && j < T && dist >= 0 && (window <= 0 || dist < window);
+            const int dist = pos - j;
+            const bool valid = row_ok && j < kv_end && dist >= 0 && (window <= 0 || dist < window);
             float x = -INFINITY;
             if (valid) {
                 x = part * scale_row;
@@ -123,24 +125,32 @@ __global__ void __launch_bounds__(kThreadsF32)
 
 template <int D>
 cudaError_t launch(const float* q, const float* k, const float* v, const float* r, const float* w, float* o,
-                   float* lse, int B, int T, int Hq, int Hkv, int window, int R, float scale, int temp_n0,
-                   cudaStream_t st) {
+                   float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int window, int R, float scale,
+                   int temp_n0, cudaStream_t st) {
     dim3 grid((T + kRows - 1) / kRows, Hq, B);
-    prefill_fp32_kernel<D><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, Hq, Hkv, window, R, scale,
-                                                         temp_n0);
+    prefill_fp32_kernel<D><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, q_off, kv_T, Hq, Hkv, window, R,
+                                                         scale, temp_n0);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
-                                float* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, int temp_n0, cudaStream_t stream) {
+                                float* o, float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
+                                int window, int R, float scale, int temp_n0, cudaStream_t stream) {
     switch (d) {
-        case 32: return launch<32>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
-        case 64: return launch<64>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
-        case 128: return launch<128>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
-        case 256: return launch<256>(q, k, v, r, w, o, lse, B, T, Hq, Hkv, window, R, scale, temp_n0, stream);
+        case 32:
+            return launch<32>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
+                              stream);
+        case 64:
+            return launch<64>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
+                              stream);
+        case 128:
+            return launch<128>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
+                              stream);
+        case 256:
+            return launch<256>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
+                              stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -54,10 +54,12 @@ constexpr int kSoftmaxRegs = 216;
 constexpr int kOtherRegs = 72;
 constexpr int kMaxDynSmem = 232448;          // 227 KB per CTA on sm_100
 
-// Reversed table: entry y <-> distance Cmax - y, Cmax = R + 255 (largest distance a
-// biased tile reaches is R + 254, smallest is -127).
+// Reversed table: entry y <-> distance Cmax - y, Cmax = R + 255.  The largest
+// distance a biased tile reaches is R + 254; the smallest a thread's run reaches is
+// -254 (a chunk of queries that starts mid-tile puts the diagonal inside a tile), so
+// the table runs down to distance -265 with zeros below 0 (those keys are masked).
 __host__ __device__ constexpr int tab_cmax(int R) { return R + 255; }
-__host__ __device__ constexpr int tab_len(int R) { return ((R + 392 + 31) / 32) * 32; }
+__host__ __device__ constexpr int tab_len(int R) { return ((R + 520 + 31) / 32) * 32; }
 __host__ __device__ constexpr int tab_stride(int R, int ncopy) {
     return tab_len(R) + (ncopy == 4 ? 8 : ncopy == 2 ? 18 : 0);
 }
@@ -127,12 +129,16 @@ __device__ __forceinline__ Item item_at(const PrefillParams& p, int k) {
     return it;
 }
 
-// First key tile and number of key tiles a query tile visits.
+// First key tile and number of key tiles the query tile with local first row i0
+// visits.  Its rows sit at positions q_off + i0 ... q_off + i0 + 127 of the sequence
+// (q_off > 0 for a chunk of queries after a cached prefix).
 __device__ __forceinline__ void kv_range(const PrefillParams& p, int i0, int& j_first, int& ntiles) {
+    const int a0 = p.q_off + i0;
     int lo = 0;
-    if (p.window > 0) lo = max(0, i0 - p.window + 1);
+    if (p.window > 0) lo = max(0, a0 - p.window + 1);
     j_first = (lo / kBN) * kBN;
-    ntiles = (i0 - j_first) / kBN + 1;
+    const int j_last = ((a0 + kBM - 1) / kBN) * kBN;   // tile holding the last row's own key
+    ntiles = (j_last - j_first) / kBN + 1;
 }
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
@@ -447,14 +453,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // context length").
             float c1 = p.scale_log2;
             if (p.temp_n0 > 1) {
-                const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
+                const int n = p.window > 0 ? min(p.q_off + i + 1, p.window) : p.q_off + i + 1;
                 if (n > p.temp_n0) c1 *= __logf(static_cast<float>(n)) * p.inv_log_n0;
             }
             const uint64_t c1x2 = f2_pack(c1, c1);
 
             for (int tt = 0; tt < ntiles; ++tt, ++tile_it) {
                 const int j0 = j_first + tt * kBN;
-                const int delta0 = i0 - j0;   // distance of (row t, key c) is delta0 + t - c
+                const int delta0 = p.q_off + i0 - j0;   // distance of (row t, key c) is delta0 + t - c
                 ok = warp_all(mbar_wait(&bars->s_full[slot], tile_it & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();

@@ -77,15 +77,18 @@ int device_info(DeviceInfo& info) {
 }
 
 // 4-D bf16 tensor map over a [B, T, H, d] tensor, box = 64 head-dim columns x
-// `rows` tokens of one head, 128-byte swizzle, zero fill outside the tensor.
-int make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int d, int rows) {
+// `rows` tokens of one head, 128-byte swizzle, zero fill outside the tensor.  With
+// T_alloc > T the tensor is the first T rows of a [B, T_alloc, H, d] allocation: rows
+// past T read as zeros.
+int make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int d, int rows, int T_alloc = 0) {
     std::string why;
     EncodeTiledFn fn = encode_fn(why);
     if (fn == nullptr) return fail(RELBIAS_ERR_CUDA, "%s", why.c_str());
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T),
                           static_cast<cuuint64_t>(B)};
+    const int Ta = T_alloc > T ? T_alloc : T;
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
-                             static_cast<cuuint64_t>(T) * H * d * 2};
+                             static_cast<cuuint64_t>(Ta) * H * d * 2};
     cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -114,13 +117,19 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 using namespace relbias;
 
-extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, const float* r, const float* w,
-                                void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
-                                float scale, int temp_n0, int dtype, void* stream) {
-    t_err.clear();
+namespace {
+
+// Prefill of T query rows at positions q_off ... q_off+T-1 against kv_T >= q_off+T
+// key/value rows (q_off = 0, kv_T = T: a whole sequence).
+int fwd_impl(const void* q, const void* k, const void* v, const float* r, const float* w, void* o, float* lse, int B,
+             int T, int q_off, int kv_T, int Hq, int Hkv, int d, int window, int R, float scale, int temp_n0,
+             int dtype, void* stream) {
     int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
     if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (q_off < 0 || static_cast<long long>(q_off) + T > kv_T)
+        return fail(RELBIAS_ERR_ARG, "need 0 <= q_off (%d) and q_off + T (%lld) <= kv_T (%d)", q_off,
+                    static_cast<long long>(q_off) + T, kv_T);
     if (B == 0 || T == 0) return RELBIAS_OK;
     if (!q || !k || !v || !r || !o) return fail(RELBIAS_ERR_ARG, "q, k, v, r and o must not be null");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
@@ -133,7 +142,7 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
             return fail(RELBIAS_ERR_UNSUPPORTED, "fp32 prefill supports d in {32, 64, 128, 256}, got %d", d);
         cudaError_t e = launch_prefill_fp32(static_cast<const float*>(q), static_cast<const float*>(k),
                                             static_cast<const float*>(v), r, w, static_cast<float*>(o), lse, B, T,
-                                            Hq, Hkv, d, window, R, scale, temp_n0, st);
+                                            q_off, kv_T, Hq, Hkv, d, window, R, scale, temp_n0, st);
         return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "fp32 prefill launch");
     }
 
@@ -148,8 +157,11 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
 
     CUtensorMap tq, tk, tv;
     if ((rc = make_map(&tq, q, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
-    if ((rc = make_map(&tk, k, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
-    if ((rc = make_map(&tv, v, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
+    // Keys and values past the chunk's last row (q_off + T - 1) are never visible;
+    // the maps end there, so tiles reaching past it read zeros, not stale cache rows
+    // (a masked key still multiplies its value row by a zero weight).
+    if ((rc = make_map(&tk, k, B, q_off + T, Hkv, d, 128, kv_T)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v, B, q_off + T, Hkv, d, 128, kv_T)) != RELBIAS_OK) return rc;
 
     PrefillParams p{};
     p.r = r;
@@ -166,6 +178,8 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     p.window = window > 0 ? window : 0;
     p.R = R;
     p.n_qt = (T + 127) / 128;
+    p.q_off = q_off;
+    p.kv_T = kv_T;
     const long long items = static_cast<long long>(p.n_qt) * B * Hkv * p.HP;
     if (items > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", items);
     p.total_items = static_cast<int>(items);
@@ -178,6 +192,23 @@ extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, con
     const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
     cudaError_t e = launch_prefill_bf16_sm100(tq, tk, tv, p, d, grid, st);
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "bf16 prefill launch");
+}
+
+}  // namespace
+
+extern "C" int relbias_attn_fwd(const void* q, const void* k, const void* v, const float* r, const float* w,
+                                void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int window, int R,
+                                float scale, int temp_n0, int dtype, void* stream) {
+    t_err.clear();
+    return fwd_impl(q, k, v, r, w, o, lse, B, T, 0, T, Hq, Hkv, d, window, R, scale, temp_n0, dtype, stream);
+}
+
+extern "C" int relbias_attn_fwd_chunk(const void* q, const void* k, const void* v, const float* r, const float* w,
+                                      void* o, float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
+                                      int window, int R, float scale, int temp_n0, int dtype, void* stream) {
+    t_err.clear();
+    return fwd_impl(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, d, window, R, scale, temp_n0, dtype,
+                    stream);
 }
 
 extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d, int window) {

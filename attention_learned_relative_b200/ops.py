@@ -33,6 +33,8 @@ _F = ctypes.c_float
 _SZ = ctypes.c_size_t
 SIGNATURES = {
     "relbias_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "relbias_attn_fwd_chunk": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                    _I, _VP]),
     "relbias_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP,
                                  _SZ, _VP]),
@@ -124,6 +126,34 @@ def attn_fwd(q, k, v, r, w, window: int, R: int, scale: float | None = None, out
     rc = lib().relbias_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
                                 B, T, Hq, Hkv, d, int(window), int(R), float(scale), int(temp_n0),
                                 _dtype_code(q), _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def attn_fwd_chunk(q, k, v, r, w, q_off: int, window: int, R: int, scale: float | None = None, out=None,
+                   lse=None, stream=None, temp_n0: int = 0):
+    """Chunked prefill: the T rows of q [B,T,Hq,d] sit at positions q_off ... q_off+T-1
+    and attend to the cache k/v [B,kv_T,Hkv,d] (kv_T >= q_off+T; rows q_off ... q_off+T-1
+    are the chunk's own keys and values).  r [B,T,Hq] fp32, w [Hq,R] fp32.  Returns
+    o [B,T,Hq,d] (fills `lse` [B,Hq,T] when given)."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,kv_T,Hkv,d]")
+    B, T, Hq, d = q.shape
+    kv_T, Hkv = k.shape[1], k.shape[2]
+    _need(k.shape[0] == B and k.shape[3] == d, "k/v shape %s does not match q %s" % (k.shape, q.shape))
+    _need(q.dtype == k.dtype == v.dtype, "q, k, v must share a dtype")
+    _need(r.shape == (B, T, Hq) and r.dtype == torch.float32, "r must be fp32 [B,T,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    for t in (q, k, v, r, w, out, lse):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out.shape == q.shape and out.dtype == q.dtype, "out must match q")
+    _need(lse is None or (lse.shape == (B, Hq, T) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq,T]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_fwd_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
+                                      B, T, int(q_off), kv_T, Hq, Hkv, d, int(window), int(R), float(scale),
+                                      int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
     _check(rc)
     return out
 

@@ -104,6 +104,27 @@ RELBIAS_API int relbias_attn_fwd(const void* q, const void* k, const void* v,
                      int dtype, void* stream);
 
 /*
+ * Chunked prefill: T new query rows at positions q_off ... q_off+T-1 of each
+ * sequence, against a key/value cache of kv_T >= q_off+T rows that already holds
+ * the prefix (rows 0 ... q_off-1) and the chunk's own keys and values (rows
+ * q_off ... q_off+T-1); rows at or past q_off+T are never read for a visible key.
+ * A serving engine processes a long prompt this way, chunk by chunk against a
+ * growing cache.  Same computation as
+ * relbias_attn_fwd for those rows: the causal mask, the window and the bias use the
+ * positions q_off + i; relbias_attn_fwd is the case q_off = 0, kv_T = T.
+ *
+ *   q [B, T, Hq, d], r [B, T, Hq], o [B, T, Hq, d], lse [B, Hq, T]: the chunk's rows
+ *   k, v [B, kv_T, Hkv, d]: the cache
+ *   q_off >= 0, q_off + T <= kv_T; other rules as for relbias_attn_fwd.
+ */
+RELBIAS_API int relbias_attn_fwd_chunk(const void* q, const void* k, const void* v,
+                     const float* r, const float* w,
+                     void* o, float* lse,
+                     int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
+                     int window, int R, float scale, int temp_n0,
+                     int dtype, void* stream);
+
+/*
  * Decode: one new query per sequence at position n_ctx-1 against a key/value
  * cache of n_ctx rows whose last row already holds that query's own key and
  * value (the 1,048,576-token context of the archdiff.com model card, "Context").

@@ -162,3 +162,30 @@ def test_paged_decode_rejects_bad_arguments(lib, kw, code):
 
 def test_paged_decode_batch_zero_is_a_no_op(lib):
     assert _paged(lib, B=0) == ops.RELBIAS_OK
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=1, T=8, q_off=16, kv_T=24, Hq=4, Hkv=2,
+             d=128, window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_BF16)
+    a.update(kw)
+    return lib.relbias_attn_fwd_chunk(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"], a["T"],
+                                      a["q_off"], a["kv_T"], a["Hq"], a["Hkv"], a["d"], a["window"], a["R"],
+                                      a["scale"], a["temp_n0"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q_off=-1), ops.RELBIAS_ERR_ARG),
+    (dict(q_off=17), ops.RELBIAS_ERR_ARG),          # q_off + T > kv_T
+    (dict(kv_T=0), ops.RELBIAS_ERR_ARG),
+    (dict(Hq=3), ops.RELBIAS_ERR_ARG),
+    (dict(k=FAKE + 2), ops.RELBIAS_ERR_ARG),
+    (dict(d=96), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_chunk_rejects_on_host(lib, kw, code):
+    assert _chunk(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_chunk_empty_is_a_no_op(lib):
+    assert _chunk(lib, T=0) == ops.RELBIAS_OK
+    assert _chunk(lib, B=0) == ops.RELBIAS_OK
