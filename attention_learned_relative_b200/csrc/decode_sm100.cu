@@ -187,14 +187,18 @@ __global__ void __launch_bounds__(kDThreads, 1)
             qb[ks][1] = hi;
         }
     }
-    // Bias feature of the two heads this thread's accumulator columns belong to.
+    // Bias feature of the two heads this thread's accumulator columns belong to, and
+    // the tables they read: per head (rank-1 form) or per sequence and head (curves of
+    // a shared bank, coefficient 1).
+    const float* wb = p.w + static_cast<size_t>(b) * p.w_bstride;
     float rs[2];
     int hcol[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int n = 2 * qq + e;
         hcol[e] = g * p.G + min(n, p.G - 1);
-        rs[e] = (n < p.G) ? __ldg(p.r + static_cast<size_t>(b) * p.Hq + g * p.G + n) * p.inv_scale : 0.0f;
+        const float coef = p.r != nullptr ? __ldg(p.r + static_cast<size_t>(b) * p.Hq + g * p.G + n) : 1.0f;
+        rs[e] = (n < p.G) ? coef * p.inv_scale : 0.0f;
     }
 
     float m_run[2] = {-INFINITY, -INFINITY};
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 if (biased) {
                     const int dist = last - key;
                     if (dist >= 0 && dist < p.R)
-                        x = fmaf(rs[col], __ldg(p.w + static_cast<size_t>(hcol[col]) * p.R + dist), x);
+                        x = fmaf(rs[col], __ldg(wb + static_cast<size_t>(hcol[col]) * p.R + dist), x);
                 }
                 bool visible = key <= last;
                 if constexpr (PAGED) visible = visible && key >= key_lo;   // aligned chunks start early
@@ -405,6 +409,32 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
 }
 
 }  // namespace
+
+namespace {
+// One thread per (sequence and head, distance): the bank's curve for the one query
+// row, sum_c rs[c] * proj[c, dist] ("Thinking Machines dropped RoPE", recipe step 2:
+// the token's coefficients times the shared functions).
+__global__ void __launch_bounds__(128) bank_curves_kernel(const float* __restrict__ rs,
+                                                          const float* __restrict__ proj, float* __restrict__ curves,
+                                                          int Hq, int C, int proj_heads, int R) {
+    const int bh = blockIdx.y;
+    const int dist = blockIdx.x * 128 + threadIdx.x;
+    if (dist >= R) return;
+    const float* coef = rs + static_cast<size_t>(bh) * C;
+    const float* bank = proj + static_cast<size_t>(proj_heads == 1 ? 0 : bh % Hq) * C * R;
+    float acc = 0.0f;
+    for (int c = 0; c < C; ++c) acc = fmaf(__ldg(coef + c), __ldg(bank + static_cast<size_t>(c) * R + dist), acc);
+    curves[static_cast<size_t>(bh) * R + dist] = acc;
+}
+}  // namespace
+
+cudaError_t launch_bank_curves(const float* rs, const float* proj, float* curves, int BH, int Hq, int C,
+                               int proj_heads, int R, cudaStream_t stream) {
+    if (BH < 1 || R < 1) return cudaSuccess;
+    dim3 grid((R + 127) / 128, BH);
+    bank_curves_kernel<<<grid, 128, 0, stream>>>(rs, proj, curves, Hq, C, proj_heads, R);
+    return cudaGetLastError();
+}
 
 int decode_num_splits(int B, int Hkv, int N, int window, int num_sms) {
     const int key_lo = window > 0 ? max(0, N - window) : 0;

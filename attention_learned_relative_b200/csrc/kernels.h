@@ -36,16 +36,26 @@ int prefill_bf16_smem_bytes(int d, int R);
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream);
 
-// fp32 SIMT prefill (prefill_fp32.cu).
+// fp32 SIMT prefill (prefill_fp32.cu).  C == 0: rank-1 bias, r [B, T, Hq] and w [Hq, R].
+// C >= 1: shared-bank bias, r [B, T, Hq, C] coefficients and w [proj_heads, C, R] curves
+// (proj_heads 1: one bank for all heads; Hq: a bank per head).
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
                                 float* o, float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
-                                int window, int R, float scale, int temp_n0, cudaStream_t stream);
+                                int window, int R, float scale, int temp_n0, int C, int proj_heads,
+                                cudaStream_t stream);
+constexpr int kMaxBankC = 16;   // functions in a shared bank
+
+// Per-(sequence, head) bias curves of the shared bank for one query row each
+// (decode_sm100.cu): curves[bh, dist] = sum_c rs[bh, c] * proj[bh % Hq or 0, c, dist].
+cudaError_t launch_bank_curves(const float* rs, const float* proj, float* curves, int BH, int Hq, int C,
+                               int proj_heads, int R, cudaStream_t stream);
 
 // bf16 split-KV decode + log-sum-exp combine (decode_sm100.cu).
 struct DecodeParams {
     const __nv_bfloat16* q;  // [B, Hq, d]
-    const float* r;          // [B, Hq]
-    const float* w;          // [Hq, R]
+    const float* r;          // [B, Hq], or nullptr: coefficient 1 (w then holds whole curves)
+    const float* w;          // [Hq, R] distance tables (w_bstride 0), or [B, Hq, R] curves
+    size_t w_bstride;        // elements between sequences' tables: 0, or Hq * R
     __nv_bfloat16* o;        // [B, Hq, d]
     float* lse;              // [B, Hq] or nullptr
     float* part;             // [B, Hq, nsplit, d + 4] workspace records

@@ -4,7 +4,9 @@
 // logit = scale * q.k + (0 <= i-j < R ? r[b,i,h] * w[h,i-j] : 0) over the causal
 // (optionally windowed) keys, softmax, weighted sum of V ("Thinking Machines
 // dropped RoPE", recipe steps 3-5; "Learned Relative-Position Bias", T5-style
-// formula).  A CTA takes 32 query rows of one (b, h); four lanes share a row and
+// formula).  The BANK instance takes the essay's shared-bank form instead: the
+// bias is sum_c r[b,i,h,c] * proj[h or 0, c, i-j], C <= 16 coefficients per token
+// and head times the bank's functions (recipe steps 1-2).  A CTA takes 32 query rows of one (b, h); four lanes share a row and
 // each holds a quarter of the head dimension (interleaved, so the four lanes read
 // four consecutive floats of a key and the eight rows of a warp share them).
 // Keys and values pass through shared memory in tiles.
@@ -21,12 +23,12 @@ namespace {
 constexpr int kRows = 32;
 constexpr int kThreadsF32 = 128;
 
-template <int D>
+template <int D, bool BANK>
 __global__ void __launch_bounds__(kThreadsF32)
     prefill_fp32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                         const float* __restrict__ r, const float* __restrict__ w, float* __restrict__ o,
                         float* __restrict__ lse, int T, int q_off, int kv_T, int Hq, int Hkv, int window, int R,
-                        float scale, int temp_n0) {
+                        float scale, int temp_n0, int C, int proj_heads) {
     constexpr int BK = D <= 128 ? 32 : 16;   // keys per shared-memory tile
     constexpr int DL = D / 4;                 // dims per lane
     __shared__ __align__(16) float ks[BK * D];
@@ -55,7 +57,16 @@ __global__ void __launch_bounds__(kThreadsF32)
         const int n = window > 0 ? min(pos + 1, window) : pos + 1;
         if (n > temp_n0) tau = static_cast<float>(log(static_cast<double>(n)) / log(static_cast<double>(temp_n0)));
     }
-    const float ri = row_ok ? tau * r[(static_cast<size_t>(b) * T + i) * Hq + h] : 0.0f;
+    const float ri = (!BANK && row_ok) ? tau * r[(static_cast<size_t>(b) * T + i) * Hq + h] : 0.0f;
+    // Shared bank: this row's coefficients (times tau) and its head's bank.
+    float rc[BANK ? kMaxBankC : 1];
+    const float* bank = w;
+    if constexpr (BANK) {
+#pragma unroll
+        for (int c = 0; c < kMaxBankC; ++c)
+            rc[c] = (row_ok && c < C) ? tau * r[((static_cast<size_t>(b) * T + i) * Hq + h) * C + c] : 0.0f;
+        bank = w + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
+    }
     const float scale_row = tau * scale;
     float m = -INFINITY, l = 0.0f;
 
@@ -93,7 +104,15 @@ __global__ void __launch_bounds__(kThreadsF32)
             float x = -INFINITY;
             if (valid) {
                 x = part * scale_row;
-                if (dist < R) x = fmaf(ri, __ldg(w + static_cast<size_t>(h) * R + dist), x);
+                if constexpr (BANK) {
+                    if (dist < R) {
+#pragma unroll
+                        for (int c = 0; c < kMaxBankC; ++c)
+                            if (c < C) x = fmaf(rc[c], __ldg(bank + static_cast<size_t>(c) * R + dist), x);
+                    }
+                } else {
+                    if (dist < R) x = fmaf(ri, __ldg(w + static_cast<size_t>(h) * R + dist), x);
+                }
             }
             s[jj] = x;
             mt = fmaxf(mt, x);
@@ -126,10 +145,14 @@ __global__ void __launch_bounds__(kThreadsF32)
 template <int D>
 cudaError_t launch(const float* q, const float* k, const float* v, const float* r, const float* w, float* o,
                    float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int window, int R, float scale,
-                   int temp_n0, cudaStream_t st) {
+                   int temp_n0, int C, int proj_heads, cudaStream_t st) {
     dim3 grid((T + kRows - 1) / kRows, Hq, B);
-    prefill_fp32_kernel<D><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, q_off, kv_T, Hq, Hkv, window, R,
-                                                         scale, temp_n0);
+    if (C > 0)
+        prefill_fp32_kernel<D, true><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, q_off, kv_T, Hq, Hkv,
+                                                                   window, R, scale, temp_n0, C, proj_heads);
+    else
+        prefill_fp32_kernel<D, false><<<grid, kThreadsF32, 0, st>>>(q, k, v, r, w, o, lse, T, q_off, kv_T, Hq, Hkv,
+                                                                    window, R, scale, temp_n0, 0, 0);
     return cudaGetLastError();
 }
 
@@ -137,20 +160,21 @@ cudaError_t launch(const float* q, const float* k, const float* v, const float* 
 
 cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, const float* r, const float* w,
                                 float* o, float* lse, int B, int T, int q_off, int kv_T, int Hq, int Hkv, int d,
-                                int window, int R, float scale, int temp_n0, cudaStream_t stream) {
+                                int window, int R, float scale, int temp_n0, int C, int proj_heads,
+                                cudaStream_t stream) {
     switch (d) {
         case 32:
-            return launch<32>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
-                              stream);
+            return launch<32>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0, C,
+                              proj_heads, stream);
         case 64:
-            return launch<64>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
-                              stream);
+            return launch<64>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0, C,
+                              proj_heads, stream);
         case 128:
-            return launch<128>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
-                              stream);
+            return launch<128>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0, C,
+                               proj_heads, stream);
         case 256:
-            return launch<256>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0,
-                              stream);
+            return launch<256>(q, k, v, r, w, o, lse, B, T, q_off, kv_T, Hq, Hkv, window, R, scale, temp_n0, C,
+                               proj_heads, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -121,9 +121,11 @@ namespace {
 
 // Prefill of T query rows at positions q_off ... q_off+T-1 against kv_T >= q_off+T
 // key/value rows (q_off = 0, kv_T = T: a whole sequence).
+// C == 0: rank-1 bias (r [B, T, Hq], w [Hq, R]); C >= 1: shared bank (r [B, T, Hq, C]
+// coefficients, w [proj_heads, C, R] functions), fp32 only.
 int fwd_impl(const void* q, const void* k, const void* v, const float* r, const float* w, void* o, float* lse, int B,
              int T, int q_off, int kv_T, int Hq, int Hkv, int d, int window, int R, float scale, int temp_n0,
-             int dtype, void* stream) {
+             int dtype, void* stream, int C = 0, int proj_heads = 0) {
     int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
     if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
@@ -142,10 +144,13 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* r, const 
             return fail(RELBIAS_ERR_UNSUPPORTED, "fp32 prefill supports d in {32, 64, 128, 256}, got %d", d);
         cudaError_t e = launch_prefill_fp32(static_cast<const float*>(q), static_cast<const float*>(k),
                                             static_cast<const float*>(v), r, w, static_cast<float*>(o), lse, B, T,
-                                            q_off, kv_T, Hq, Hkv, d, window, R, scale, temp_n0, st);
+                                            q_off, kv_T, Hq, Hkv, d, window, R, scale, temp_n0, C, proj_heads, st);
         return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "fp32 prefill launch");
     }
 
+    if (C > 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED,
+                    "the shared-bank bias runs on the fp32 prefill path only (bf16 prefill takes the rank-1 form)");
     if (d != 64 && d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill supports d in {64, 128}, got %d", d);
     if (R > 2048 || prefill_bf16_table_copies(d, R) == 0)
         return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
@@ -211,6 +216,31 @@ extern "C" int relbias_attn_fwd_chunk(const void* q, const void* k, const void* 
                     stream);
 }
 
+namespace relbias {
+namespace {
+int check_bank(int C, int proj_heads, int Hq) {
+    if (C < 1 || C > kMaxBankC) return fail(RELBIAS_ERR_ARG, "C (%d) must be in [1, %d]", C, kMaxBankC);
+    if (proj_heads != 1 && proj_heads != Hq)
+        return fail(RELBIAS_ERR_ARG, "proj_heads (%d) must be 1 or Hq (%d)", proj_heads, Hq);
+    return RELBIAS_OK;
+}
+size_t bank_curve_bytes(int B, int Hq, int R) {
+    const size_t b = static_cast<size_t>(B) * Hq * std::max(R, 0) * sizeof(float);
+    return (b + 255) / 256 * 256;
+}
+}  // namespace
+}  // namespace relbias
+
+extern "C" int relbias_attn_fwd_bank(const void* q, const void* k, const void* v, const float* rs, const float* proj,
+                                     void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
+                                     int window, int R, float scale, int temp_n0, int dtype, void* stream) {
+    t_err.clear();
+    const int rc = check_bank(C, proj_heads, Hq);
+    if (rc != RELBIAS_OK) return rc;
+    return fwd_impl(q, k, v, rs, proj, o, lse, B, T, 0, T, Hq, Hkv, d, window, R, scale, temp_n0, dtype, stream, C,
+                    proj_heads);
+}
+
 extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d, int window) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || n_ctx < 1 || d < 1) return 0;
     DeviceInfo dev;
@@ -219,17 +249,18 @@ extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int
     return decode_workspace_bytes(B, Hq, nsplit, d);
 }
 
-extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const void* v_cache, const float* r,
-                                   const float* w, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d,
-                                   int window, int R, float scale, int temp_n0, int dtype, void* workspace,
-                                   size_t ws_bytes, void* stream) {
-    t_err.clear();
+namespace {
+// Contiguous-cache decode.  w_bstride == 0: rank-1 tables w [Hq, R] times r [B, Hq];
+// w_bstride == Hq * R: per-sequence curves w [B, Hq, R] with coefficient 1 (r unused).
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* r, const float* w,
+                size_t w_bstride, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d, int window, int R,
+                float scale, int temp_n0, int dtype, void* workspace, size_t ws_bytes, void* stream) {
     int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
     if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
     if (B == 0) return RELBIAS_OK;
     if (n_ctx < 1) return fail(RELBIAS_ERR_ARG, "n_ctx (%d) must be >= 1", n_ctx);
-    if (!q || !k_cache || !v_cache || !r || !o || !workspace)
+    if (!q || !k_cache || !v_cache || (w_bstride == 0 && !r) || !o || !workspace)
         return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, r, o and workspace must not be null");
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace))
         return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, o and workspace must be 16-byte aligned");
@@ -245,8 +276,9 @@ extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const voi
 
     DecodeParams p{};
     p.q = static_cast<const __nv_bfloat16*>(q);
-    p.r = r;
+    p.r = w_bstride == 0 ? r : nullptr;
     p.w = w;
+    p.w_bstride = w_bstride;
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.part = static_cast<float*>(workspace);
@@ -282,6 +314,50 @@ extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const voi
     if ((rc = make_map(&tv, v_cache, B, n_ctx, Hkv, d, kChunk)) != RELBIAS_OK) return rc;
     cudaError_t e = launch_decode_bf16(tk, tv, p, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "decode launch");
+}
+}  // namespace
+
+extern "C" int relbias_attn_decode(const void* q, const void* k_cache, const void* v_cache, const float* r,
+                                   const float* w, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d,
+                                   int window, int R, float scale, int temp_n0, int dtype, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+    t_err.clear();
+    return decode_impl(q, k_cache, v_cache, r, w, 0, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale, temp_n0, dtype,
+                       workspace, ws_bytes, stream);
+}
+
+extern "C" size_t relbias_attn_decode_bank_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d, int window,
+                                                          int R) {
+    const size_t base = relbias_attn_decode_workspace_size(B, Hq, Hkv, n_ctx, d, window);
+    if (base == 0 || R < 0) return 0;
+    return bank_curve_bytes(B, Hq, R) + base;
+}
+
+extern "C" int relbias_attn_decode_bank(const void* q, const void* k_cache, const void* v_cache, const float* rs,
+                                        const float* proj, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv,
+                                        int d, int C, int proj_heads, int window, int R, float scale, int temp_n0,
+                                        int dtype, void* workspace, size_t ws_bytes, void* stream) {
+    t_err.clear();
+    int rc = check_bank(C, proj_heads, Hq);
+    if (rc != RELBIAS_OK) return rc;
+    if ((rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, proj)) != RELBIAS_OK) return rc;
+    if (B == 0) return RELBIAS_OK;
+    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports bf16 only");
+    if (d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports d == 128, got %d", d);
+    if (!rs || !aligned4(rs)) return fail(RELBIAS_ERR_ARG, "rs is null or not 4-byte aligned");
+    if (!workspace || !aligned16(workspace)) return fail(RELBIAS_ERR_ARG, "workspace is null or not 16-byte aligned");
+    const size_t cb = bank_curve_bytes(B, Hq, R);
+    if (ws_bytes < cb) return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes cannot hold the %zu bytes of curves",
+                                   ws_bytes, cb);
+    float* curves = static_cast<float*>(workspace);
+    if (R > 0) {
+        const cudaError_t e = launch_bank_curves(rs, proj, curves, B * Hq, Hq, C, proj_heads, R,
+                                                 static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "bank curve launch");
+    }
+    return decode_impl(q, k_cache, v_cache, nullptr, curves, static_cast<size_t>(Hq) * R, o, lse, B, n_ctx, Hq, Hkv,
+                       d, window, R, scale, temp_n0, dtype, static_cast<char*>(workspace) + cb, ws_bytes - cb,
+                       stream);
 }
 
 namespace relbias {
@@ -400,7 +476,7 @@ extern "C" int relbias_device_status(int reset) {
     return static_cast<int>(v);
 }
 
-extern "C" int relbias_version(void) { return 200; }
+extern "C" int relbias_version(void) { return 300; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"

@@ -43,6 +43,11 @@ SIGNATURES = {
     "relbias_attn_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode_paged": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
                                        _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
+    "relbias_attn_fwd_bank": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                   _I, _VP]),
+    "relbias_attn_decode_bank_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "relbias_attn_decode_bank": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                      _I, _VP, _SZ, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_version": (_I, []),
@@ -258,6 +263,73 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, r, w, window: 
                                          block_table.shape[1], int(max_seq_len), Hq, Hkv, d, int(window), int(R),
                                          float(scale), int(temp_n0), _dtype_code(q), _ptr(workspace), ws_bytes,
                                          _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def _bank_shape(proj, C_from_rs: int, Hq: int, R: int) -> int:
+    """proj_heads of a bank tensor [proj_heads, C, R] (proj_heads 1 or Hq)."""
+    _need(proj is not None and proj.dim() == 3 and proj.dtype == torch.float32, "proj must be fp32 [heads,C,R]")
+    _need(proj.shape[1] == C_from_rs and proj.shape[2] == R and proj.shape[0] in (1, Hq),
+          "proj must be [1 or Hq, C, R] = [*, %d, %d], got %s" % (C_from_rs, R, tuple(proj.shape)))
+    return int(proj.shape[0])
+
+
+def attn_fwd_bank(q, k, v, rs, proj, window: int, R: int, scale: float | None = None, out=None, lse=None,
+                  stream=None, temp_n0: int = 0):
+    """Prefill with the shared-bank bias sum_c rs[b,i,h,c] * proj[h or 0, c, i-j].
+    q [B,T,Hq,d], k/v [B,T,Hkv,d] fp32 (the bank form runs on the fp32 path),
+    rs [B,T,Hq,C] fp32, proj [1 or Hq, C, R] fp32.  Returns o [B,T,Hq,d]."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(rs.dim() == 4 and rs.shape[:3] == (B, T, Hq) and rs.dtype == torch.float32, "rs must be fp32 [B,T,Hq,C]")
+    C = int(rs.shape[3])
+    proj_heads = _bank_shape(proj, C, Hq, R)
+    for t in (q, k, v, rs, proj, out, lse):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(lse is None or (lse.shape == (B, Hq, T) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq,T]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_fwd_bank(_ptr(q), _ptr(k), _ptr(v), _ptr(rs), _ptr(proj), _ptr(out), _ptr(lse),
+                                     B, T, Hq, Hkv, d, C, proj_heads, int(window), int(R), float(scale),
+                                     int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def decode_bank_workspace_size(B: int, Hq: int, Hkv: int, n_ctx: int, d: int, window: int, R: int) -> int:
+    """Bytes of scratch attn_decode_bank needs (curves plus split partials)."""
+    return int(lib().relbias_attn_decode_bank_workspace_size(B, Hq, Hkv, n_ctx, d, window, R))
+
+
+def attn_decode_bank(q, k_cache, v_cache, rs, proj, window: int, R: int, scale: float | None = None, out=None,
+                     lse=None, workspace=None, stream=None, temp_n0: int = 0):
+    """Decode with the shared-bank bias.  q [B,Hq,d] bf16, caches [B,n_ctx,Hkv,d]
+    bf16, rs [B,Hq,C] fp32, proj [1 or Hq, C, R] fp32.  Returns o [B,Hq,d]."""
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "q [B,Hq,d], cache [B,N,Hkv,d]")
+    B, Hq, d = q.shape
+    _, N, Hkv, _ = k_cache.shape
+    _need(rs.dim() == 3 and rs.shape[:2] == (B, Hq) and rs.dtype == torch.float32, "rs must be fp32 [B,Hq,C]")
+    C = int(rs.shape[2])
+    proj_heads = _bank_shape(proj, C, Hq, R)
+    for t in (q, k_cache, v_cache, rs, proj, out, lse, workspace):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(lse is None or (lse.shape == (B, Hq) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq]")
+    need = decode_bank_workspace_size(B, Hq, Hkv, N, d, window, R)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_decode_bank(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(rs), _ptr(proj), _ptr(out),
+                                        _ptr(lse), B, N, Hq, Hkv, d, C, proj_heads, int(window), int(R),
+                                        float(scale), int(temp_n0), _dtype_code(q), _ptr(workspace), ws_bytes,
+                                        _stream_handle(stream, q.device))
     _check(rc)
     return out
 

@@ -25,7 +25,7 @@ _W1 = 0xBB67AE85
 _MASK = 0xFFFFFFFF
 
 # Tensor ids: one key per input of the attention call.
-TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "r": 4, "w": 5, "bank": 6, "rs": 7}
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "r": 4, "w": 5, "bank": 6, "rs": 7, "proj": 8}
 
 
 def _mulhilo(a: torch.Tensor, m: int):

@@ -34,6 +34,7 @@ class Workload:
     decode: bool = False
     qk_std: float = 1.0   # Q and K are drawn as N(0, qk_std^2)
     page_size: int = 0    # decode only: > 0 stores the cache as shuffled pages of this many rows
+    bank_C: int = 0       # > 0: shared-bank bias with this many functions (rs, proj inputs)
 
     @property
     def scale(self) -> float:
@@ -82,6 +83,10 @@ WORKLOADS = {
         # block table is a seeded random permutation (scattered physical pages).
         Workload("global_decode_paged_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0,
                  R=1024, seed=4, dtype="bf16", decode=True, page_size=256),
+        # The same decode step with the essay's shared-bank bias: 16 functions of
+        # distance shared by all heads, 16 coefficients per (token, head).
+        Workload("global_decode_bank_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0,
+                 R=1024, seed=4, dtype="bf16", decode=True, bank_C=16),
     ]
 }
 
@@ -111,6 +116,13 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
     v = synth.normal((B, T, wl.Hkv, wl.d), s, "v", dtype=dt, device=device)
     w = synth.normal((wl.Hq, wl.R), s, "w", std=0.5, device=device)
     x = {"q": q, "k": k, "v": v, "r": r, "w": w}
+    if wl.bank_C > 0:
+        # Shared bank: rs ~ N(0, 1/C) coefficients and proj ~ N(0, 0.5^2) functions, so a
+        # curve value sum_c rs[c] proj[c, dist] has the spread of r * w (std 0.5).
+        C = wl.bank_C
+        shape = (B, wl.Hq, C) if wl.decode else (B, T, wl.Hq, C)
+        x["rs"] = synth.normal(shape, s, "rs", std=1.0 / math.sqrt(C), device=device)
+        x["proj"] = synth.normal((1, C, wl.R), s, "proj", std=0.5, device=device)
     if wl.decode and wl.page_size > 0:
         if T % wl.page_size != 0:
             raise ValueError("paged workload needs T (%d) divisible by page_size (%d)" % (T, wl.page_size))

@@ -198,6 +198,10 @@ def step_fn(wl, ops, workspace):
             ops.attn_decode_paged(x["q"], x["k_pages"], x["v_pages"], x["table"], x["lens"], x["r"], x["w"],
                                   wl.window, wl.R, wl.T, wl.scale, out=x["o"], lse=x["lse"], workspace=workspace,
                                   stream=stream)
+    elif wl.decode and wl.bank_C > 0:
+        def step(x, stream):
+            ops.attn_decode_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], wl.window, wl.R, wl.scale, out=x["o"],
+                                 lse=x["lse"], workspace=workspace, stream=stream)
     elif wl.decode:
         def step(x, stream):
             ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
@@ -231,8 +235,12 @@ def cpu_baseline(wl, x, budget_s):
             k_sl, v_sl = logical_cache(x, b, kv)
             k_sl, v_sl = k_sl[None].cpu(), v_sl[None].cpu()
             q = x["q"][b, heads].float().cpu()
-            r = x["r"][b, heads].cpu().reshape(G, 1)
-            proj = x["w"][heads].cpu().reshape(G, 1, wl.R)
+            if wl.bank_C > 0:
+                r = x["rs"][b, heads].cpu()              # [G, C]
+                proj = x["proj"].cpu()                   # [1, C, R], shared by the heads
+            else:
+                r = x["r"][b, heads].cpu().reshape(G, 1)
+                proj = x["w"][heads].cpu().reshape(G, 1, wl.R)
             req = np.array([(0, hl, wl.T - 1) for hl in range(G)], dtype=np.int64)
             t0 = time.perf_counter()
             O.attn_rows(q, r, proj, k_sl, v_sl, req, G, wl.window, wl.R, wl.scale)
@@ -305,6 +313,8 @@ def run_ours(args, wl, peaks, peaks_kind):
     if wl.decode:
         if wl.page_size > 0:
             nbytes = ops.decode_paged_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
+        elif wl.bank_C > 0:
+            nbytes = ops.decode_bank_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window, wl.R)
         else:
             nbytes = ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
@@ -342,7 +352,10 @@ def run_ours(args, wl, peaks, peaks_kind):
     e2e = None
     if not args.no_e2e:
         x = sets[0]
-        names_in = ["q", "r"] if wl.decode else ["q", "k", "v", "r", "w"]
+        if wl.decode:
+            names_in = ["q", "rs"] if wl.bank_C > 0 else ["q", "r"]
+        else:
+            names_in = ["q", "k", "v", "r", "w"]
         host_in = {n: x[n].cpu().pin_memory() for n in names_in}
         host_out = torch.empty(x["o"].shape, dtype=x["o"].dtype, pin_memory=True)
         bi = sum(t.numel() * t.element_size() for t in host_in.values())
@@ -380,7 +393,8 @@ def run_ours(args, wl, peaks, peaks_kind):
             peak = float(peaks["hbm_gbs"])
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "traffic": traffic, "peak_source": peaks_kind + " hbm_gbs (copy)",
-                    "kernel": "decode_splitkv_kernel + decode_combine_kernel",
+                    "kernel": ("bank_curves_kernel + " if wl.bank_C > 0 else "")
+                    + "decode_splitkv_kernel + decode_combine_kernel",
                     "algorithmic_bytes_per_launch": per_step}
         else:
             unit = "TFLOP/s"
@@ -414,12 +428,13 @@ def run_ours(args, wl, peaks, peaks_kind):
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
                        "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
                        **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
+                       **({"bias": "shared bank, C=%d functions" % wl.bank_C} if wl.bank_C > 0 else {}),
                        "parallelism": "dp%d (batch shards, no collective)" % world,
                        "l2": ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6))
                        if nsets > 1 else "per-step input %.0f MB > L2" % (step_bytes / 1e6)},
             "roofline": roof,
             "clocks": clocks.summary(),
-            "gpu_launches": steps * (2 if wl.decode else 1),
+            "gpu_launches": steps * ((3 if wl.bank_C > 0 else 2) if wl.decode else 1),
             "kernel_status": status,
         }
         if e2e is not None:

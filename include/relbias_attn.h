@@ -219,6 +219,47 @@ RELBIAS_API int relbias_attn_decode_paged(const void* q, const void* k_pages, co
                         int window, int R, float scale, int temp_n0,
                         int dtype, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Shared-bank bias.  The essay's recipe ("Thinking Machines dropped RoPE", steps
+ * 1-2) keeps a small bank of C learned functions of distance, shared by the
+ * heads of a layer, and gives every token and head C coefficients from a
+ * projection; the bias is the coefficients times the bank:
+ *
+ *   bias[j] = sum_c rs[b,i,h,c] * proj[h', c, i-j]   if 0 <= i-j < R, else 0
+ *
+ * with h' = 0 (one bank for all heads, proj_heads = 1) or h' = h (a bank per
+ * head, proj_heads = Hq).  The rank-1 form of relbias_attn_fwd is the case
+ * C = 1, proj_heads = Hq.  1 <= C <= 16.
+ *
+ * relbias_attn_fwd_bank: prefill, RELBIAS_FP32 only (the bf16 tensor-core
+ * kernel takes the rank-1 form and returns RELBIAS_ERR_UNSUPPORTED here).
+ *   rs   [B, T, Hq, C]          fp32
+ *   proj [proj_heads, C, R]     fp32   (may be NULL if R == 0)
+ *   other arguments as for relbias_attn_fwd.
+ *
+ * relbias_attn_decode_bank: decode as relbias_attn_decode, with
+ *   rs   [B, Hq, C]             fp32   the new token's coefficients
+ *   proj [proj_heads, C, R]     fp32
+ * The call first writes each (sequence, head) curve sum_c rs[c] * proj[c, :]
+ * (B * Hq * R floats) into the front of `workspace`; the split-KV kernels then
+ * read those curves.  ws_bytes must be at least
+ * relbias_attn_decode_bank_workspace_size(...).
+ */
+RELBIAS_API int relbias_attn_fwd_bank(const void* q, const void* k, const void* v,
+                     const float* rs, const float* proj,
+                     void* o, float* lse,
+                     int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
+                     int window, int R, float scale, int temp_n0,
+                     int dtype, void* stream);
+RELBIAS_API size_t relbias_attn_decode_bank_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d,
+                                          int window, int R);
+RELBIAS_API int relbias_attn_decode_bank(const void* q, const void* k_cache, const void* v_cache,
+                     const float* rs, const float* proj,
+                     void* o, float* lse,
+                     int B, int n_ctx, int Hq, int Hkv, int d, int C, int proj_heads,
+                     int window, int R, float scale, int temp_n0,
+                     int dtype, void* workspace, size_t ws_bytes, void* stream);
+
 /* Description of the last failed call on this thread ("" if none).  The string
  * stays valid until the next library call on the same thread. */
 RELBIAS_API const char* relbias_last_error(void);

@@ -48,7 +48,7 @@ def test_binding_argument_counts_match_header():
 
 
 def test_version(lib):
-    assert ops.version() >= 200
+    assert ops.version() >= 300
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
@@ -189,3 +189,53 @@ def test_chunk_rejects_on_host(lib, kw, code):
 def test_chunk_empty_is_a_no_op(lib):
     assert _chunk(lib, T=0) == ops.RELBIAS_OK
     assert _chunk(lib, B=0) == ops.RELBIAS_OK
+
+
+def _fwd_bank(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, rs=FAKE, proj=FAKE, o=FAKE, lse=None, B=1, T=8, Hq=4, Hkv=2, d=64, C=16,
+             proj_heads=1, window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_FP32)
+    a.update(kw)
+    return lib.relbias_attn_fwd_bank(a["q"], a["k"], a["v"], a["rs"], a["proj"], a["o"], a["lse"], a["B"], a["T"],
+                                     a["Hq"], a["Hkv"], a["d"], a["C"], a["proj_heads"], a["window"], a["R"],
+                                     a["scale"], a["temp_n0"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(C=0), ops.RELBIAS_ERR_ARG),
+    (dict(C=17), ops.RELBIAS_ERR_ARG),
+    (dict(proj_heads=2), ops.RELBIAS_ERR_ARG),       # neither 1 nor Hq
+    (dict(rs=None), ops.RELBIAS_ERR_ARG),
+    (dict(proj=None), ops.RELBIAS_ERR_ARG),
+    (dict(dtype=ops.RELBIAS_BF16, d=128), ops.RELBIAS_ERR_UNSUPPORTED),   # bank runs on the fp32 path
+    (dict(d=48), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_fwd_bank_rejects_on_host(lib, kw, code):
+    assert _fwd_bank(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def _dec_bank(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, rs=FAKE, proj=FAKE, o=FAKE, lse=None, B=2, N=100, Hq=8, Hkv=1, d=128, C=16,
+             proj_heads=1, window=0, R=16, scale=0.1, temp_n0=0, dtype=ops.RELBIAS_BF16, ws=FAKE, ws_bytes=64)
+    a.update(kw)
+    return lib.relbias_attn_decode_bank(a["q"], a["k"], a["v"], a["rs"], a["proj"], a["o"], a["lse"], a["B"],
+                                        a["N"], a["Hq"], a["Hkv"], a["d"], a["C"], a["proj_heads"], a["window"],
+                                        a["R"], a["scale"], a["temp_n0"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(C=0), ops.RELBIAS_ERR_ARG),
+    (dict(proj_heads=3), ops.RELBIAS_ERR_ARG),
+    (dict(rs=None), ops.RELBIAS_ERR_ARG),
+    (dict(ws=None), ops.RELBIAS_ERR_ARG),
+    (dict(ws_bytes=64), ops.RELBIAS_ERR_ARG),          # 2*8*16 floats of curves do not fit 64 bytes
+    (dict(dtype=ops.RELBIAS_FP32), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(d=64), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_decode_bank_rejects_on_host(lib, kw, code):
+    assert _dec_bank(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_decode_bank_empty_batch(lib):
+    assert _dec_bank(lib, B=0) == ops.RELBIAS_OK
