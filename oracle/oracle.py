@@ -53,6 +53,12 @@ def _load():
                       ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int64,
                       ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_num_threads.restype = ctypes.c_int
+        fb = lib.oracle_attn_bwd
+        fb.restype = ctypes.c_int
+        fb.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                       ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                       ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int64,
+                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         _lib = lib
     return _lib
 
@@ -163,6 +169,41 @@ def attn_prefill(q, k, v, r, w, window: int, R: int, scale: float, rows=None, te
     if rows is not None:
         return o, lse
     return o.reshape(B, T, Hq, d), lse.reshape(B, T, Hq).transpose(0, 2, 1).copy()
+
+
+def attn_backward(q, k, v, r, w, dout, window: int, R: int, scale: float, temp_n0: int = 0):
+    """Gradients of the prefill (relbias_oracle.c, oracle_attn_bwd, states the steps).
+
+    Shapes as attn_prefill, plus dout [B, T, Hq, d] = dL/dO.  Returns a dict of fp64
+    arrays: dq [B,T,Hq,d], dk and dv [B,T,Hkv,d], dr shaped like r, dw shaped like w.
+    """
+    lib = _load()
+    q = _f32(q)
+    k = _f32(k)
+    v = _f32(v)
+    r_in = _f32(r)
+    w_in = _f32(w)
+    dout = _f32(dout)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != k.shape or dout.shape != q.shape:
+        raise ValueError("q %s, k %s, v %s, dout %s do not fit" % (q.shape, k.shape, v.shape, dout.shape))
+    proj = np.ascontiguousarray(_tables(w_in, Hq, R))
+    Hp, C, _ = proj.shape
+    if r_in.size != B * T * Hq * C:
+        raise ValueError("r has %d values, expected B*T*Hq*C = %d" % (r_in.size, B * T * Hq * C))
+    rs = np.ascontiguousarray(r_in.reshape(B, T, Hq, C))
+    dq = np.zeros((B, T, Hq, d))
+    dk = np.zeros((B, T, Hkv, d))
+    dv = np.zeros((B, T, Hkv, d))
+    drs = np.zeros((B, T, Hq, C))
+    dproj = np.zeros((Hp, C, max(R, 0)))
+    rc = lib.oracle_attn_bwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, rs.ctypes.data, proj.ctypes.data, Hp, C,
+                             dout.ctypes.data, B, T, Hq, Hkv, d, int(window), int(R), float(scale), int(temp_n0),
+                             dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, drs.ctypes.data, dproj.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd rejected its arguments")
+    return {"dq": dq, "dk": dk, "dv": dv, "dr": drs.reshape(r_in.shape), "dw": dproj.reshape(w_in.shape)}
 
 
 def attn_decode(q, k_cache, v_cache, r, w, window: int, R: int, scale: float, temp_n0: int = 0):

@@ -178,6 +178,156 @@ int oracle_attn_rows(const float* q_rows, const float* rs_rows,
     return status;
 }
 
+/* Gradients of the whole forward pass (the backward pass), in fp64.
+ *
+ * Loss-independent form: given dout = dL/dO for every output row, return dL/d of
+ * every input.  For one row (b, h, i) with logits l_j = tau * (scale * q.k_j +
+ * bias_j) over j in A_i, p_j = exp(l_j - LSE_i) and O_i = sum_j p_j v_j (the
+ * forward above), the chain rule gives, step by step:
+ *   dp_j   = dout_i . v_j                       (O is linear in p)
+ *   D_i    = sum_j p_j dp_j  (= dout_i . O_i)
+ *   dl_j   = p_j (dp_j - D_i)                   (softmax Jacobian)
+ *   dq_i  += dl_j * tau * scale * k_j           (l_j through the dot product)
+ *   dk_j  += dl_j * tau * scale * q_i
+ *   dv_j  += p_j * dout_i
+ *   dbias  = dl_j * tau, for 0 <= i-j < R       (step 5: the bias adds to the logit)
+ *   drs[i,c]        += dbias * proj[c, i-j]     (step 2: curve = sum_c rs[c] proj[c, .])
+ *   dproj[h', c, i-j] += dbias * rs[i,c]
+ * Key/value gradients sum over the query heads of their group; a bank shared by
+ * all heads (Hp == 1) sums over every head.  tau depends only on the number of
+ * visible keys, not on any input, so it is a constant factor here.
+ *
+ *   q, dout [B, T, Hq, d]; k, v [B, T, Hkv, d]; rs [B, T, Hq, C]; proj [Hp, C, R]
+ *   dq [B, T, Hq, d]; dk, dv [B, T, Hkv, d]; drs [B, T, Hq, C]; dproj [Hp, C, R]
+ *   (all outputs fp64, overwritten).
+ * Heads run in parallel (OpenMP), each into private key/value and table
+ * buffers that are summed afterwards in a fixed order.
+ * Returns 0, or -1 on a bad argument or allocation failure.
+ */
+int oracle_attn_bwd(const float* q, const float* k, const float* v, const float* rs,
+                    const float* proj, int Hp, int C, const float* dout,
+                    int B, int64_t T, int Hq, int Hkv, int d,
+                    int64_t window, int64_t R, double scale, int64_t temp_n0,
+                    double* dq, double* dk, double* dv, double* drs, double* dproj)
+{
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || C <= 0 || R < 0) return -1;
+    if (Hq % Hkv != 0 || !(Hp == 1 || Hp == Hq)) return -1;
+    const int G = Hq / Hkv;
+    const int64_t kv_stride = (int64_t)Hkv * d;
+    memset(dq, 0, sizeof(double) * (size_t)B * T * Hq * d);
+    memset(dk, 0, sizeof(double) * (size_t)B * T * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * T * Hkv * d);
+    memset(drs, 0, sizeof(double) * (size_t)B * T * Hq * C);
+    memset(dproj, 0, sizeof(double) * (size_t)Hp * C * (R > 0 ? R : 0));
+
+    /* private per-head buffers: dk/dv contributions [Hq][T][d], table grads [Hq][C][R] */
+    double* dk_h = (double*)calloc((size_t)Hq * T * d, sizeof(double));
+    double* dv_h = (double*)calloc((size_t)Hq * T * d, sizeof(double));
+    double* dp_h = (double*)calloc((size_t)Hq * C * (R > 0 ? R : 1), sizeof(double));
+    if (!dk_h || !dv_h || !dp_h) { free(dk_h); free(dv_h); free(dp_h); return -1; }
+    int status = 0;
+
+    for (int b = 0; b < B; ++b) {
+        memset(dk_h, 0, sizeof(double) * (size_t)Hq * T * d);
+        memset(dv_h, 0, sizeof(double) * (size_t)Hq * T * d);
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int h = 0; h < Hq; ++h) {
+            const int64_t g = h / G;
+            const float* table = proj + (Hp == 1 ? 0 : h) * (int64_t)C * R;
+            double* logit = (double*)malloc((size_t)T * sizeof(double));
+            double* curve = (double*)malloc((size_t)(R > 0 ? R : 1) * sizeof(double));
+            double* o_row = (double*)malloc((size_t)d * sizeof(double));
+            if (!logit || !curve || !o_row) {
+                free(logit); free(curve); free(o_row);
+#pragma omp atomic write
+                status = -1;
+                continue;
+            }
+            for (int64_t i = 0; i < T; ++i) {
+                const float* qi = q + ((b * T + i) * Hq + h) * (int64_t)d;
+                const float* doi = dout + ((b * T + i) * Hq + h) * (int64_t)d;
+                const float* rsi = rs + ((b * T + i) * Hq + h) * (int64_t)C;
+                for (int64_t dd = 0; dd < R; ++dd) {
+                    double acc = 0.0;
+                    for (int c = 0; c < C; ++c) acc += (double)rsi[c] * (double)table[(int64_t)c * R + dd];
+                    curve[dd] = acc;
+                }
+                int64_t j_lo = 0;
+                if (window > 0 && i - window + 1 > 0) j_lo = i - window + 1;
+                const int64_t n = i - j_lo + 1;
+                double tau = 1.0;
+                if (temp_n0 > 1 && n > temp_n0) tau = log((double)n) / log((double)temp_n0);
+                /* forward recomputed: logits, max, sum, O */
+                double m = -INFINITY;
+                for (int64_t j = j_lo; j <= i; ++j) {
+                    const float* kj = k + (b * T + j) * kv_stride + g * d;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c) dot += (double)qi[c] * (double)kj[c];
+                    const int64_t dist = i - j;
+                    const double bias = (dist < R) ? curve[dist] : 0.0;
+                    logit[j] = tau * (scale * dot + bias);
+                    if (logit[j] > m) m = logit[j];
+                }
+                double den = 0.0;
+                for (int64_t j = j_lo; j <= i; ++j) den += exp(logit[j] - m);
+                const double lse = m + log(den);
+                for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+                for (int64_t j = j_lo; j <= i; ++j) {
+                    const double p = exp(logit[j] - lse);
+                    const float* vj = v + (b * T + j) * kv_stride + g * d;
+                    for (int c = 0; c < d; ++c) o_row[c] += p * (double)vj[c];
+                }
+                double D = 0.0;
+                for (int c = 0; c < d; ++c) D += (double)doi[c] * o_row[c];
+                /* backward through softmax, dot products and bias */
+                double* dqi = dq + ((b * T + i) * Hq + h) * (int64_t)d;
+                double* drsi = drs + ((b * T + i) * Hq + h) * (int64_t)C;
+                for (int64_t j = j_lo; j <= i; ++j) {
+                    const float* kj = k + (b * T + j) * kv_stride + g * d;
+                    const float* vj = v + (b * T + j) * kv_stride + g * d;
+                    const double p = exp(logit[j] - lse);
+                    double dp = 0.0;
+                    for (int c = 0; c < d; ++c) dp += (double)doi[c] * (double)vj[c];
+                    const double dl = p * (dp - D);
+                    double* dkj = dk_h + ((int64_t)h * T + j) * d;
+                    double* dvj = dv_h + ((int64_t)h * T + j) * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqi[c] += dl * tau * scale * (double)kj[c];
+                        dkj[c] += dl * tau * scale * (double)qi[c];
+                        dvj[c] += p * (double)doi[c];
+                    }
+                    const int64_t dist = i - j;
+                    if (dist < R) {
+                        const double dbias = dl * tau;
+                        double* dph = dp_h + (int64_t)h * C * R;
+                        for (int c = 0; c < C; ++c) {
+                            drsi[c] += dbias * (double)table[(int64_t)c * R + dist];
+                            dph[(int64_t)c * R + dist] += dbias * (double)rsi[c];
+                        }
+                    }
+                }
+            }
+            free(logit); free(curve); free(o_row);
+        }
+        /* sum the heads of each group into the key/value gradients, in head order */
+        for (int h = 0; h < Hq; ++h) {
+            const int64_t g = h / G;
+            for (int64_t j = 0; j < T; ++j)
+                for (int c = 0; c < d; ++c) {
+                    dk[((b * T + j) * Hkv + g) * d + c] += dk_h[((int64_t)h * T + j) * d + c];
+                    dv[((b * T + j) * Hkv + g) * d + c] += dv_h[((int64_t)h * T + j) * d + c];
+                }
+        }
+    }
+    /* table gradients: per head, or summed over all heads for a shared bank */
+    for (int h = 0; h < Hq; ++h) {
+        double* dst = dproj + (Hp == 1 ? 0 : h) * (int64_t)C * R;
+        for (int64_t x = 0; x < (int64_t)C * R; ++x) dst[x] += dp_h[(int64_t)h * C * R + x];
+    }
+    free(dk_h); free(dv_h); free(dp_h);
+    return status;
+}
+
 /* Threads the OpenMP loop above would use. */
 int oracle_num_threads(void)
 {
