@@ -45,6 +45,14 @@ cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, 
                                 cudaStream_t stream);
 constexpr int kMaxBankC = 16;   // functions in a shared bank
 
+// Backward pass on CUDA cores (backward_fp32.cu): dq [B,T,Hq,d], dk/dv [B,T,Hkv,d], dr
+// [B,T,Hq], dw [Hq,R] (zeroed here, then accumulated), all fp32; q, k, v, o, dout in
+// bf16 (bf16 == true) or fp32; dvec [B,Hq,T] scratch for D_i = dout_i . o_i.
+cudaError_t launch_backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* r,
+                            const float* w, const void* o, const float* lse, const void* dout, float* dq, float* dk,
+                            float* dv, float* dr, float* dw, float* dvec, int B, int T, int Hq, int Hkv, int window,
+                            int R, float scale, int temp_n0, cudaStream_t stream);
+
 // Per-(sequence, head) bias curves of the shared bank for one query row each
 // (decode_sm100.cu): curves[bh, dist] = sum_c rs[bh, c] * proj[bh % Hq or 0, c, dist].
 cudaError_t launch_bank_curves(const float* rs, const float* proj, float* curves, int BH, int Hq, int C,

@@ -17,6 +17,7 @@
 #include "decode_sm100.cu"
 #include "prefill_fp32.cu"
 #include "prefill_sm100.cu"
+#include "backward_fp32.cu"
 
 namespace relbias {
 namespace {
@@ -459,6 +460,41 @@ extern "C" int relbias_attn_decode_paged(const void* q, const void* k_pages, con
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "paged decode launch");
 }
 
+extern "C" size_t relbias_attn_bwd_workspace_size(int B, int T, int Hq) {
+    if (B < 0 || T < 0 || Hq < 1) return 0;
+    const size_t n = static_cast<size_t>(B) * Hq * T * sizeof(float);
+    return n < 16 ? 16 : n;
+}
+
+extern "C" int relbias_attn_bwd(const void* q, const void* k, const void* v, const float* r, const float* w,
+                                const void* o, const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                                float* dr, float* dw, int B, int T, int Hq, int Hkv, int d, int window, int R,
+                                float scale, int temp_n0, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+    t_err.clear();
+    int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0 || T == 0) return RELBIAS_OK;
+    if (!q || !k || !v || !r || !o || !lse || !dout || !dq || !dk || !dv || !dr || (R > 0 && !dw) || !workspace)
+        return fail(RELBIAS_ERR_ARG, "q, k, v, r, o, lse, dout, dq, dk, dv, dr, dw (R > 0) and workspace must not be "
+                                     "null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return fail(RELBIAS_ERR_ARG, "q, k, v, o, dout, dq, dk, dv and workspace must be 16-byte aligned");
+    if (!aligned4(r) || !aligned4(lse) || !aligned4(dr) || (dw && !aligned4(dw)))
+        return fail(RELBIAS_ERR_ARG, "r, lse, dr and dw must be 4-byte aligned");
+    if (d != 32 && d != 64 && d != 128 && d != 256)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "the backward pass supports d in {32, 64, 128, 256}, got %d", d);
+    if (R > 32768) return fail(RELBIAS_ERR_UNSUPPORTED, "the backward pass stages R <= 32768 table gradients");
+    if (ws_bytes < relbias_attn_bwd_workspace_size(B, T, Hq))
+        return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes,
+                    relbias_attn_bwd_workspace_size(B, T, Hq));
+    const cudaError_t e = launch_backward(dtype == RELBIAS_BF16, d, q, k, v, r, w, o, lse, dout, dq, dk, dv, dr, dw,
+                                          static_cast<float*>(workspace), B, T, Hq, Hkv, window > 0 ? window : 0, R,
+                                          scale, temp_n0 > 1 ? temp_n0 : 0, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "backward launch");
+}
+
 extern "C" const char* relbias_last_error(void) { return t_err.c_str(); }
 
 extern "C" int relbias_device_status(int reset) {
@@ -476,7 +512,7 @@ extern "C" int relbias_device_status(int reset) {
     return static_cast<int>(v);
 }
 
-extern "C" int relbias_version(void) { return 300; }
+extern "C" int relbias_version(void) { return 400; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"

@@ -48,6 +48,8 @@ SIGNATURES = {
     "relbias_attn_decode_bank_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode_bank": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                       _I, _VP, _SZ, _VP]),
+    "relbias_attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
+    "relbias_attn_bwd": (_I, [_VP] * 13 + [_I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_version": (_I, []),
@@ -332,6 +334,44 @@ def attn_decode_bank(q, k_cache, v_cache, rs, proj, window: int, R: int, scale: 
                                         _stream_handle(stream, q.device))
     _check(rc)
     return out
+
+
+def attn_bwd(q, k, v, r, w, o, lse, dout, window: int, R: int, scale: float | None = None, stream=None,
+             temp_n0: int = 0, workspace=None, grads=None):
+    """Backward pass of attn_fwd.  q/o/dout [B,T,Hq,d], k/v [B,T,Hkv,d] (bf16 or fp32),
+    r [B,T,Hq] and w [Hq,R] fp32, lse [B,Hq,T] fp32 (the forward's).  Returns a dict of
+    fp32 gradients dq, dk, dv (shapes of q, k, v), dr [B,T,Hq] and dw [Hq,R] (written
+    into `grads` when a dict of such tensors is given)."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(o.shape == q.shape and dout.shape == q.shape, "o and dout must have q's shape")
+    _need(q.dtype == k.dtype == v.dtype == o.dtype == dout.dtype, "q, k, v, o, dout must share a dtype")
+    _need(r.shape == (B, T, Hq) and r.dtype == torch.float32, "r must be fp32 [B,T,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    _need(lse.shape == (B, Hq, T) and lse.dtype == torch.float32, "lse must be fp32 [B,Hq,T]")
+    for t in (q, k, v, r, w, o, lse, dout, workspace):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = grads if grads is not None else {
+        "dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32), "dv": torch.empty(v.shape, **f32),
+        "dr": torch.empty(r.shape, **f32), "dw": torch.empty((Hq, max(R, 0)), **f32)}
+    for name, like in (("dq", q), ("dk", k), ("dv", v), ("dr", r)):
+        _need(g[name].shape == like.shape and g[name].dtype == torch.float32 and g[name].is_contiguous(),
+              "%s must be a contiguous fp32 tensor of shape %s" % (name, tuple(like.shape)))
+    need = int(lib().relbias_attn_bwd_workspace_size(B, T, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(o), _ptr(lse), _ptr(dout),
+                                _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dr"]),
+                                _ptr(g["dw"]) if R > 0 else None, B, T, Hq, Hkv, d, int(window), int(R),
+                                float(scale), int(temp_n0), _dtype_code(q), _ptr(workspace), ws_bytes,
+                                _stream_handle(stream, q.device))
+    _check(rc)
+    return g
 
 
 def device_status(reset: bool = True) -> int:

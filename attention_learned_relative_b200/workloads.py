@@ -35,6 +35,7 @@ class Workload:
     qk_std: float = 1.0   # Q and K are drawn as N(0, qk_std^2)
     page_size: int = 0    # decode only: > 0 stores the cache as shuffled pages of this many rows
     bank_C: int = 0       # > 0: shared-bank bias with this many functions (rs, proj inputs)
+    backward: bool = False  # prefill only: the step is the backward pass (dout input, gradients out)
 
     @property
     def scale(self) -> float:
@@ -54,8 +55,11 @@ class Workload:
         return W * (W + 1) // 2 + (T - W) * W
 
     def masked_flops(self) -> int:
-        """2 flops per multiply-add of QK^T and PV over attended pairs only."""
-        return 4 * self.d * self.attended_pairs() * self.B * self.Hq
+        """2 flops per multiply-add of QK^T and PV over attended pairs only.  For a
+        backward workload: the five products of the backward pass (QK^T recomputed,
+        dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q), 2.5 times the forward."""
+        per_pair = 10 * self.d if self.backward else 4 * self.d
+        return per_pair * self.attended_pairs() * self.B * self.Hq
 
     def kv_bytes(self) -> int:
         """Bytes of K and V a decode step must stream (the attended cache rows)."""
@@ -87,6 +91,9 @@ WORKLOADS = {
         # distance shared by all heads, 16 coefficients per (token, head).
         Workload("global_decode_bank_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0,
                  R=1024, seed=4, dtype="bf16", decode=True, bank_C=16),
+        # The backward pass of the local-layer prefill (the pages train the model).
+        Workload("local_backward_bf16", B=2, T=8192, Hq=32, Hkv=4, d=128, window=512, R=512,
+                 seed=1, dtype="bf16", backward=True),
     ]
 }
 
@@ -116,6 +123,8 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
     v = synth.normal((B, T, wl.Hkv, wl.d), s, "v", dtype=dt, device=device)
     w = synth.normal((wl.Hq, wl.R), s, "w", std=0.5, device=device)
     x = {"q": q, "k": k, "v": v, "r": r, "w": w}
+    if wl.backward:
+        x["dout"] = synth.normal((B, T, wl.Hq, wl.d), s, "bank", dtype=dt, device=device)
     if wl.bank_C > 0:
         # Shared bank: rs ~ N(0, 1/C) coefficients and proj ~ N(0, 0.5^2) functions, so a
         # curve value sum_c rs[c] proj[c, dist] has the spread of r * w (std 0.5).

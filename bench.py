@@ -185,6 +185,15 @@ def make_sets(wl, nsets, device):
         if wl.decode:
             x["o"] = torch.empty_like(x["q"])
             x["lse"] = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
+        elif wl.backward:
+            # The forward's O and LSE are inputs of the backward: computed once, untimed.
+            from attention_learned_relative_b200 import ops
+            x["lse"] = torch.empty(wl.B, wl.Hq, wl.T, dtype=torch.float32, device=device)
+            x["o"] = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, lse=x["lse"])
+            f32 = dict(dtype=torch.float32, device=device)
+            x["g"] = {"dq": torch.empty(x["q"].shape, **f32), "dk": torch.empty(x["k"].shape, **f32),
+                      "dv": torch.empty(x["v"].shape, **f32), "dr": torch.empty(x["r"].shape, **f32),
+                      "dw": torch.empty(wl.Hq, wl.R, **f32)}
         else:
             x["o"] = torch.empty_like(x["q"])
             x["lse"] = torch.empty(wl.B, wl.Hq, wl.T, dtype=torch.float32, device=device)
@@ -206,11 +215,22 @@ def step_fn(wl, ops, workspace):
         def step(x, stream):
             ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
                             lse=x["lse"], workspace=workspace, stream=stream)
+    elif wl.backward:
+        def step(x, stream):
+            ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], x["o"], x["lse"], x["dout"], wl.window, wl.R,
+                         wl.scale, stream=stream, workspace=workspace, grads=x["g"])
     else:
         def step(x, stream):
             ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
                          lse=x["lse"], stream=stream)
     return step
+
+
+def step_outputs(wl, x):
+    """The device tensors a step produces (read back to the host in the e2e measurement)."""
+    if wl.backward:
+        return [x["g"][n] for n in ("dq", "dk", "dv", "dr", "dw")]
+    return [x["o"]]
 
 
 def cpu_baseline(wl, x, budget_s):
@@ -250,6 +270,32 @@ def cpu_baseline(wl, x, budget_s):
         return nbytes / t_all / 1e9, O.num_threads(), \
             "%d (sequence, kv-head) groups of %s, all %d query heads each over the full cache (%.1f s)" % (
                 groups, wl.name, G, t_all), t_all
+
+    if wl.backward:
+        # The oracle's backward over a prefix of sequence 0 (all heads): causal, so the
+        # prefix is a complete sub-problem.  Its length is sized to the time budget.
+        def run(n):
+            args = [x[t][:1, :n].cpu() for t in ("q", "k", "v", "r")]
+            t0 = time.perf_counter()
+            O.attn_backward(args[0], args[1], args[2], args[3], x["w"].cpu(), x["dout"][:1, :n].cpu(), wl.window,
+                            wl.R, wl.scale)
+            return time.perf_counter() - t0
+
+        def pairs(n):
+            W = wl.window
+            return n * (n + 1) // 2 if (W <= 0 or W >= n) else W * (W + 1) // 2 + (n - W) * W
+
+        n0 = min(256, wl.T)
+        t_small = max(run(n0), 1e-4)
+        per_pair = t_small / pairs(n0)
+        n = n0
+        while n < wl.T and pairs(min(wl.T, 2 * n)) * per_pair <= budget_s:
+            n = min(wl.T, 2 * n)
+        dt = run(n)
+        fl = 10.0 * wl.d * pairs(n) * wl.Hq
+        return fl / dt / 1e12, O.num_threads(), \
+            "backward of the first %d tokens of sequence 0 of %s, all %d heads (%.3g masked GFLOP, %.1f s)" % (
+                n, wl.name, wl.Hq, fl / 1e9, dt), dt
 
     k_cpu = x["k"].cpu()
     v_cpu = x["v"].cpu()
@@ -305,11 +351,16 @@ def run_ours(args, wl, peaks, peaks_kind):
         step_bytes = wl.kv_bytes()
     else:
         step_bytes = (2 * wl.B * wl.T * wl.Hq * wl.d + 2 * wl.B * wl.T * wl.Hkv * wl.d) * esz
+        if wl.backward:   # o and dout in, fp32 gradients out
+            step_bytes += 2 * wl.B * wl.T * wl.Hq * wl.d * esz + 4 * wl.B * wl.T * (wl.Hq + 2 * wl.Hkv) * wl.d
     l2 = 126 * 2 ** 20
     nsets = 1 if step_bytes > 3 * l2 else int(math.ceil(3 * l2 / step_bytes)) + 1
     wl, _ = rank_workload(wl, rank, world)
     sets = make_sets(wl, nsets, dev)
     workspace = None
+    if wl.backward:
+        workspace = torch.empty(max(16, ops.lib().relbias_attn_bwd_workspace_size(wl.B, wl.T, wl.Hq)),
+                                dtype=torch.uint8, device=dev)
     if wl.decode:
         if wl.page_size > 0:
             nbytes = ops.decode_paged_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
@@ -354,19 +405,23 @@ def run_ours(args, wl, peaks, peaks_kind):
         x = sets[0]
         if wl.decode:
             names_in = ["q", "rs"] if wl.bank_C > 0 else ["q", "r"]
+        elif wl.backward:
+            names_in = ["q", "k", "v", "r", "w", "o", "lse", "dout"]
         else:
             names_in = ["q", "k", "v", "r", "w"]
         host_in = {n: x[n].cpu().pin_memory() for n in names_in}
-        host_out = torch.empty(x["o"].shape, dtype=x["o"].dtype, pin_memory=True)
+        dev_out = step_outputs(wl, x)
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in dev_out]
         bi = sum(t.numel() * t.element_size() for t in host_in.values())
-        bo = host_out.numel() * host_out.element_size()
+        bo = sum(t.numel() * t.element_size() for t in host_out)
         e2e_steps = max(3, min(steps, 50))
 
         def e2e_step():
             for n, t in host_in.items():
                 x[n].copy_(t, non_blocking=True)
             step(x, stream)
-            host_out.copy_(x["o"], non_blocking=True)
+            for h_, d_ in zip(host_out, dev_out):
+                h_.copy_(d_, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -402,15 +457,17 @@ def run_ours(args, wl, peaks, peaks_kind):
             value = per_step * world / (ms_step * 1e-3) / 1e12
             achieved = per_step / (ms_step * 1e-3) / 1e12
             peak = float(peaks["bf16_tflops"])
-            if wl.dtype != "bf16":
+            if wl.dtype != "bf16" or wl.backward:
                 # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
                 peak = 148 * 128 * 2 * 1.965e9 / 1e12
-            roof = {"bound": "tensor" if wl.dtype == "bf16" else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            tensor = wl.dtype == "bf16" and not wl.backward
+            roof = {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
-                    "peak_source": (peaks_kind + " bf16_tflops (burst)") if wl.dtype == "bf16"
+                    "peak_source": (peaks_kind + " bf16_tflops (burst)") if tensor
                     else "fp32 FMA units x max clock",
                     "frac_of_datasheet_2250": achieved / 2250.0,
-                    "kernel": "prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel",
+                    "kernel": "bwd_dq_kernel + bwd_dkv_kernel" if wl.backward
+                    else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel"),
                     "algorithmic_flops_per_launch": per_step}
         result = {
             "metric": METRIC,
@@ -429,12 +486,13 @@ def run_ours(args, wl, peaks, peaks_kind):
                        "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
                        **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
                        **({"bias": "shared bank, C=%d functions" % wl.bank_C} if wl.bank_C > 0 else {}),
+                       **({"pass": "backward (dq, dk, dv, dr, dw)"} if wl.backward else {}),
                        "parallelism": "dp%d (batch shards, no collective)" % world,
                        "l2": ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6))
                        if nsets > 1 else "per-step input %.0f MB > L2" % (step_bytes / 1e6)},
             "roofline": roof,
             "clocks": clocks.summary(),
-            "gpu_launches": steps * ((3 if wl.bank_C > 0 else 2) if wl.decode else 1),
+            "gpu_launches": steps * ((3 if wl.bank_C > 0 else 2) if wl.decode else (2 if wl.backward else 1)),
             "kernel_status": status,
         }
         if e2e is not None:

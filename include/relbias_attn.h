@@ -260,6 +260,36 @@ RELBIAS_API int relbias_attn_decode_bank(const void* q, const void* k_cache, con
                      int window, int R, float scale, int temp_n0,
                      int dtype, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Backward pass of relbias_attn_fwd (rank-1 bias): given dout = dL/dO, the
+ * gradients of every input.  The pages train this model but print no backward;
+ * these are the derivatives of the forward definition above.  With logits
+ * l_j = tau_i * (scale * q_i.k_j + bias_ij), p_j = exp(l_j - lse_i) and
+ * D_i = dout_i . o_i:
+ *   dl_j = p_j * (dout_i . v_j - D_i)
+ *   dq_i = tau_i * scale * sum_j dl_j k_j     dk_j = sum over (h, i) of tau_i * scale * dl_j q_i
+ *   dv_j = sum over (h, i) of p_j dout_i      dr_i = sum_j tau_i dl_j w[h, i-j]
+ *   dw[h, d] = sum_i tau_i dl_(i, i-d) r_i    (bias terms only where 0 <= i-j < R)
+ *
+ *   q, o, dout [B, T, Hq, d]  dtype     k, v [B, T, Hkv, d]  dtype
+ *   r [B, T, Hq], w [Hq, R]   fp32      lse [B, Hq, T] fp32: the forward's log-sum-exp
+ *   dq [B, T, Hq, d], dk and dv [B, T, Hkv, d], dr [B, T, Hq], dw [Hq, R]: fp32
+ *     outputs, overwritten (dw may be NULL if R == 0)
+ *   workspace: at least relbias_attn_bwd_workspace_size(B, T, Hq) bytes of
+ *     caller-owned device scratch (D_i per row), 16-byte aligned.
+ * o and lse must be the forward's outputs for the same inputs.  dtype
+ * RELBIAS_BF16 or RELBIAS_FP32 (fp32 arithmetic on CUDA cores either way);
+ * d in {32, 64, 128, 256}; R <= 32768; other rules as for relbias_attn_fwd.
+ */
+RELBIAS_API size_t relbias_attn_bwd_workspace_size(int B, int T, int Hq);
+RELBIAS_API int relbias_attn_bwd(const void* q, const void* k, const void* v,
+                     const float* r, const float* w,
+                     const void* o, const float* lse, const void* dout,
+                     float* dq, float* dk, float* dv, float* dr, float* dw,
+                     int B, int T, int Hq, int Hkv, int d,
+                     int window, int R, float scale, int temp_n0,
+                     int dtype, void* workspace, size_t ws_bytes, void* stream);
+
 /* Description of the last failed call on this thread ("" if none).  The string
  * stays valid until the next library call on the same thread. */
 RELBIAS_API const char* relbias_last_error(void);

@@ -48,7 +48,7 @@ def test_binding_argument_counts_match_header():
 
 
 def test_version(lib):
-    assert ops.version() >= 300
+    assert ops.version() >= 400
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
@@ -239,3 +239,34 @@ def test_decode_bank_rejects_on_host(lib, kw, code):
 
 def test_decode_bank_empty_batch(lib):
     assert _dec_bank(lib, B=0) == ops.RELBIAS_OK
+
+
+def _bwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, dr=FAKE,
+             dw=FAKE, B=1, T=8, Hq=4, Hkv=2, d=64, window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_BF16,
+             ws=FAKE, ws_bytes=16)
+    a.update(kw)
+    return lib.relbias_attn_bwd(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["dout"], a["dq"], a["dk"],
+                                a["dv"], a["dr"], a["dw"], a["B"], a["T"], a["Hq"], a["Hkv"], a["d"], a["window"],
+                                a["R"], a["scale"], a["temp_n0"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lse=None), ops.RELBIAS_ERR_ARG),
+    (dict(dw=None), ops.RELBIAS_ERR_ARG),             # R > 0 needs dw
+    (dict(dout=FAKE + 4), ops.RELBIAS_ERR_ARG),
+    (dict(Hq=3), ops.RELBIAS_ERR_ARG),
+    (dict(dtype=5), ops.RELBIAS_ERR_ARG),
+    (dict(d=96), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(R=40000), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(ws_bytes=16), ops.RELBIAS_ERR_ARG),          # B*Hq*T floats = 128 bytes needed
+])
+def test_bwd_rejects_on_host(lib, kw, code):
+    assert _bwd(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_bwd_empty_and_workspace_size(lib):
+    assert _bwd(lib, T=0) == ops.RELBIAS_OK
+    assert ops.lib().relbias_attn_bwd_workspace_size(2, 100, 8) == 2 * 100 * 8 * 4
+    assert ops.lib().relbias_attn_bwd_workspace_size(0, 100, 8) == 16

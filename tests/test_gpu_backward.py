@@ -1,0 +1,104 @@
+"""GPU parity of the backward pass (relbias_attn_bwd) against the fp64 oracle's
+gradients (oracle_attn_bwd, itself pinned by finite differences of the forward).
+
+The kernel gets O and LSE from the oracle's forward (stored in the kernel's dtype),
+as a training step would get them from the forward pass.  Tolerance, relative to the
+largest reference gradient of each tensor: 1e-4 for fp32 (fp32 sums of up to a few
+thousand terms); 1e-2 for bf16, where O is stored in bf16 and D_i = dout_i . o_i
+inherits its 2^-9 relative rounding.
+"""
+import math
+
+import pytest
+import torch
+
+from attention_learned_relative_b200 import ops, synth
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    ops.device_status(reset=True)
+    yield
+    assert ops.device_status(reset=True) == 0, "a kernel wait timed out"
+
+
+def _inputs(dtype, B, T, Hq, Hkv, d, R, seed):
+    dev = "cuda"
+    return {
+        "q": synth.normal((B, T, Hq, d), seed, "q", dtype=dtype, device=dev),
+        "k": synth.normal((B, T, Hkv, d), seed, "k", dtype=dtype, device=dev),
+        "v": synth.normal((B, T, Hkv, d), seed, "v", dtype=dtype, device=dev),
+        "r": synth.normal((B, T, Hq), seed, "r", device=dev),
+        "w": synth.normal((Hq, R), seed, "w", std=0.5, device=dev),
+        "dout": synth.normal((B, T, Hq, d), seed, "bank", dtype=dtype, device=dev),
+    }
+
+
+def _check(g, ref, tol, what):
+    for name in ("dq", "dk", "dv", "dr", "dw"):
+        a = g[name].double().cpu()
+        b = torch.as_tensor(ref[name]).reshape(a.shape)
+        if b.numel() == 0:
+            continue
+        scale = b.abs().max().item()
+        err = (a - b).abs().max().item()
+        assert err <= tol * scale + 1e-7, "%s %s: max err %.3e vs max |ref| %.3e" % (what, name, err, scale)
+
+
+CASES = [
+    # dtype,          B, T,    Hq, Hkv, d,   window, R,   temp_n0
+    (torch.float32, 1, 100, 4, 2, 64, 0, 50, 0),
+    (torch.float32, 2, 150, 4, 1, 32, 40, 60, 0),       # window, GQA group 4, ragged tiles
+    (torch.float32, 1, 300, 2, 2, 128, 0, 300, 100),    # temperature
+    (torch.float32, 1, 97, 4, 4, 256, 16, 20, 0),       # d = 256
+    (torch.float32, 1, 64, 2, 1, 64, 0, 0, 0),          # R = 0: no bias, no dw
+    (torch.bfloat16, 1, 256, 8, 2, 128, 0, 128, 0),
+    (torch.bfloat16, 1, 1024, 8, 2, 128, 512, 512, 0),  # the local-layer shape over 32 tiles
+]
+
+
+@pytest.mark.parametrize("dtype,B,T,Hq,Hkv,d,window,R,temp_n0", CASES)
+def test_backward_parity(dtype, B, T, Hq, Hkv, d, window, R, temp_n0):
+    x = _inputs(dtype, B, T, Hq, Hkv, d, R, seed=T + d + R)
+    scale = 1.0 / math.sqrt(d)
+    o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), window,
+                                    R, scale, temp_n0=temp_n0)
+    o = torch.as_tensor(o_ref).to(dtype).cuda()
+    lse = torch.as_tensor(lse_ref).float().cuda()
+    g = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], window, R, scale, temp_n0=temp_n0)
+    torch.cuda.synchronize()
+    ref = O.attn_backward(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), x["dout"].cpu(),
+                          window, R, scale, temp_n0=temp_n0)
+    _check(g, ref, 1e-4 if dtype == torch.float32 else 1e-2,
+           "backward %s" % ((dtype, B, T, Hq, Hkv, d, window, R, temp_n0),))
+
+
+def test_backward_after_the_bf16_forward():
+    """A training step's own pair: the tensor-core forward's O and LSE feed the backward."""
+    B, T, Hq, Hkv, d, window, R = 1, 640, 8, 2, 128, 512, 512
+    x = _inputs(torch.bfloat16, B, T, Hq, Hkv, d, R, seed=3)
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], window, R, lse=lse)
+    g = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], window, R)
+    torch.cuda.synchronize()
+    ref = O.attn_backward(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), x["dout"].cpu(),
+                          window, R, 1.0 / math.sqrt(d))
+    _check(g, ref, 2e-2, "backward after forward")
+
+
+def test_backward_is_deterministic_except_dw():
+    """dq, dk, dv and dr are written without atomics: bitwise repeatable."""
+    x = _inputs(torch.float32, 1, 200, 4, 2, 64, 64, seed=11)
+    o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), 0, 64,
+                                    0.125)
+    o = torch.as_tensor(o_ref).float().cuda()
+    lse = torch.as_tensor(lse_ref).float().cuda()
+    g1 = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], 0, 64, 0.125)
+    g2 = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], 0, 64, 0.125)
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv", "dr"):
+        assert torch.equal(g1[name], g2[name]), name
+    assert (g1["dw"] - g2["dw"]).abs().max().item() <= 1e-5 * g1["dw"].abs().max().item()
