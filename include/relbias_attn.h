@@ -55,7 +55,7 @@ extern "C" {
 
 #define RELBIAS_OK               0
 #define RELBIAS_ERR_ARG         -1  /* null pointer, bad shape, misalignment, bad scale   */
-#define RELBIAS_ERR_UNSUPPORTED -2  /* valid request this build or device cannot serve    */
+#define RELBIAS_ERR_UNSUPPORTED -2  /* valid request the library or device cannot serve   */
 #define RELBIAS_ERR_CUDA        -3  /* a CUDA runtime call or kernel launch failed        */
 
 /* Bytes of the static scratch behind relbias_attn_decode_noalloc (8 MiB). */
