@@ -1,0 +1,31 @@
+"""The benchmark's CPU-baseline leg (the oracle timed on a bounded sample) on small
+copies of every workload kind: prefill, decode, paged decode, shared-bank decode and
+the backward pass.  No GPU: inputs are drawn on the CPU."""
+import os
+import sys
+from dataclasses import replace
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from attention_learned_relative_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_cpu_baseline_runs_on_every_workload_kind(name):
+    wl = WORKLOADS[name]
+    small = replace(wl, B=min(wl.B, 2), T=min(wl.T, 512), R=min(wl.R, 256),
+                    window=min(wl.window, 128) if wl.window > 0 else wl.window)
+    x = make_inputs(small, device="cpu")
+    rate, cores, desc, dt = bench.cpu_baseline(small, x, 0.05)
+    assert rate > 0 and cores >= 1 and dt > 0
+    assert small.name in desc
+
+
+def test_backward_flops_are_two_and_a_half_forwards():
+    fwd = WORKLOADS["local_prefill_bf16"]
+    bwd = WORKLOADS["local_backward_bf16"]
+    assert bwd.masked_flops() * 2 == fwd.masked_flops() * 5
