@@ -29,3 +29,21 @@ def test_backward_flops_are_two_and_a_half_forwards():
     fwd = WORKLOADS["local_prefill_bf16"]
     bwd = WORKLOADS["local_backward_bf16"]
     assert bwd.masked_flops() * 2 == fwd.masked_flops() * 5
+
+
+@pytest.mark.parametrize("T,window", [(1, 0), (7, 0), (100, 0), (100, 1), (100, 17), (100, 100), (100, 250)])
+def test_attended_pairs_match_a_brute_force_count(T, window):
+    """The FLOP count the benchmark divides by: pairs (i, j) with 0 <= i - j and, for a
+    window, i - j < window, counted one by one."""
+    wl = replace(WORKLOADS["tiny_local_fp32"], T=T, window=window, B=3, Hq=5, d=16)
+    brute = sum(1 for i in range(T) for j in range(T) if 0 <= i - j and (window <= 0 or i - j < window))
+    assert wl.attended_pairs() == brute
+    assert wl.masked_flops() == 4 * 16 * brute * 3 * 5
+
+
+def test_decode_bytes_are_the_attended_cache_rows():
+    wl = WORKLOADS["global_decode_bf16"]
+    assert wl.attended_pairs() == wl.T
+    assert wl.kv_bytes() == 2 * wl.B * wl.Hkv * wl.T * wl.d * 2
+    win = replace(wl, window=512)
+    assert win.kv_bytes() == 2 * wl.B * wl.Hkv * 512 * wl.d * 2
