@@ -35,6 +35,7 @@ CASES = [
     (2, 11, 4, 2, 8, 5, 7, 1, 4, 0),      # window, GQA
     (1, 12, 2, 2, 8, 0, 12, 3, 1, 0),     # shared bank of 3 functions
     (1, 14, 2, 1, 8, 0, 6, 1, 2, 4),      # temperature: tau > 1 for rows seeing > 4 keys
+    (1, 10, 2, 1, 8, 4, 8, 2, 2, 0),      # a bank of 2 functions per head, window
 ]
 
 
