@@ -47,3 +47,19 @@ def test_decode_bytes_are_the_attended_cache_rows():
     assert wl.kv_bytes() == 2 * wl.B * wl.Hkv * wl.T * wl.d * 2
     win = replace(wl, window=512)
     assert win.kv_bytes() == 2 * wl.B * wl.Hkv * 512 * wl.d * 2
+
+
+def test_committed_ncu_summaries_describe_the_current_kernels():
+    """Every ncu summary under profiles/ names the digest of the CUDA sources it was taken
+    on; it must be the digest of the sources in the tree."""
+    import re
+    prof = os.path.join(ROOT, "profiles")
+    found = 0
+    for name in sorted(os.listdir(prof)):
+        if not name.startswith("ncu_"):
+            continue
+        m = re.search(r"source_sha256:\s*([0-9a-f]+)", open(os.path.join(prof, name)).read())
+        assert m, name
+        assert m.group(1) == bench.source_digest(), name
+        found += 1
+    assert found >= 3
