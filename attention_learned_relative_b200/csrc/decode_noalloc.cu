@@ -13,11 +13,14 @@
 // In host code the array's name is only a host-side stand-in for the symbol, not
 // a device address: handing it to a kernel would fault, or on systems where the
 // GPU can reach host memory silently use the wrong memory.  The real device
-// address is looked up with cudaGetSymbolAddress, once per device, with that
-// device current, on the first call made on that device.
+// address is looked up with cudaGetSymbolAddress, with the caller's device and
+// context current, on every call.  The lookup is a host-side table query that
+// allocates nothing; doing it per call keeps the address right after a
+// cudaDeviceReset (which unloads and reloads the library's device image) and when
+// a caller switches between contexts of the same device.  The first call on a
+// device may load the library's device image there (lazy module loading), so it
+// should come before any stream capture.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "relbias_attn.h"
 
@@ -25,28 +28,19 @@ namespace relbias {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = RELBIAS_DECODE_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // The shared scratch: partial (max, sum, output) records of the split-KV kernel.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (looked up once).
+// Device address of g_noalloc_scratch in the current context.
 int noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) return fail(RELBIAS_ERR_UNSUPPORTED, "device index %d out of range", dev);
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
-        g_noalloc_ptr[dev] = p;
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+        cudaGetLastError();   // do not leave the failed lookup pending for the caller's next check
+        return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(decode scratch)");
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return RELBIAS_OK;
 }
 
@@ -59,21 +53,23 @@ extern "C" int relbias_attn_decode_noalloc(const void* q, const void* k_cache, c
                                            void* stream) {
     using namespace relbias;
     t_err.clear();
-    // Argument errors first, exactly as the regular entry point reports them.
-    int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
-    if (rc != RELBIAS_OK) return rc;
-    if (B == 0)
-        return relbias_attn_decode(q, k_cache, v_cache, r, w, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale,
-                                   temp_n0, dtype, nullptr, 0, stream);
-    void* ws = nullptr;
-    if ((rc = noalloc_scratch(&ws)) != RELBIAS_OK) return rc;
-    const size_t need = relbias_attn_decode_workspace_size(B, Hq, Hkv, n_ctx, d, window);
+    // Argument and device checks first, with the same codes and messages as
+    // relbias_attn_decode: a bad call never reaches the symbol lookup.
+    bool nothing_to_do = false;
+    DeviceInfo dev;
+    int rc = decode_check_args(q, k_cache, v_cache, r, w, 0, o, lse, B, n_ctx, Hq, Hkv, d, R, scale, dtype,
+                               false, nullptr, &nothing_to_do, &dev);
+    if (rc != RELBIAS_OK || nothing_to_do) return rc;
+    const int nsplit = decode_num_splits(B, Hkv, n_ctx, window > 0 ? window : 0, dev.sms);
+    const size_t need = decode_workspace_bytes(B, Hq, nsplit, d);
     if (need > kNoAllocScratchBytes)
         return fail(RELBIAS_ERR_UNSUPPORTED,
                     "this decode needs %zu bytes of scratch, more than the %zu-byte static scratch of "
                     "relbias_attn_decode_noalloc; call relbias_attn_decode with a workspace instead",
                     need, kNoAllocScratchBytes);
-    // The split partials are written before they are read: nothing needs clearing.
+    void* ws = nullptr;
+    if ((rc = noalloc_scratch(&ws)) != RELBIAS_OK) return rc;
+    // Every split partial is written before the combine reads it: nothing needs clearing.
     return relbias_attn_decode(q, k_cache, v_cache, r, w, o, lse, B, n_ctx, Hq, Hkv, d, window, R, scale, temp_n0,
                                dtype, ws, kNoAllocScratchBytes, stream);
 }

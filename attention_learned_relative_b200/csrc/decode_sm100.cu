@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
+            int issued = 0;   // chunks whose copies were issued
             for (int li = 0; li < nloc; ++li) {
                 const int st = li % kDStages;
                 const uint32_t ph = (li / kDStages) & 1;
@@ -160,11 +161,13 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 tma_load_4d(base + kBoxBytes, &tm_k, &bars->full[st], 64, g, row, seq);
                 tma_load_4d(base + 2 * kBoxBytes, &tm_v, &bars->full[st], 0, g, row, seq);
                 tma_load_4d(base + 3 * kBoxBytes, &tm_v, &bars->full[st], 64, g, row, seq);
+                issued = li + 1;
             }
-            // Do not leave while copies into this CTA's shared memory are in flight.
-            int dummy = 0;
-            for (int li = max(0, nloc - kDStages); li < nloc; ++li)
-                mbar_wait(&bars->full[li % kDStages], (li / kDStages) & 1, &dummy);
+            // Do not leave while copies into this CTA's shared memory are in flight: wait
+            // for the last phase issued on each stage (earlier ones completed before their
+            // stage was refilled).
+            for (int li = max(0, issued - kDStages); li < issued; ++li)
+                mbar_drain_wait(&bars->full[li % kDStages], (li / kDStages) & 1);
         }
         return;
     }
@@ -197,7 +200,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
     for (int e = 0; e < 2; ++e) {
         const int n = 2 * qq + e;
         hcol[e] = g * p.G + min(n, p.G - 1);
-        const float coef = p.r != nullptr ? __ldg(p.r + static_cast<size_t>(b) * p.Hq + g * p.G + n) : 1.0f;
+        // Columns n >= G are padding heads: their feature is never read (with G < 8
+        // the address would belong to the next group, or lie past the end of r).
+        const float coef =
+            (p.r != nullptr && n < p.G) ? __ldg(p.r + static_cast<size_t>(b) * p.Hq + g * p.G + n) : 1.0f;
         rs[e] = (n < p.G) ? coef * p.inv_scale : 0.0f;
     }
 

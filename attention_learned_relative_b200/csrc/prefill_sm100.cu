@@ -80,6 +80,7 @@ struct Bars {
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_final[2];
+    uint64_t tab_sync[2];             // per slot: its four softmax warps meet around table staging
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
@@ -142,6 +143,16 @@ __device__ __forceinline__ void kv_range(const PrefillParams& p, int i0, int& j_
 }
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// The four softmax warps of a slot meet: each arrives once (after its own shared-memory
+// writes, which the arrival releases), then waits for the phase with a bounded wait.
+__device__ __forceinline__ bool tab_meet(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = warp_all(mbar_wait(bar, phase & 1, abort_flag));
+    ++phase;
+    return ok;
+}
 
 template <int D>
 __device__ __forceinline__ void issue_qk(bool leader, uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr,
@@ -255,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->p_full[s], kBM / 32);   // one arrival per softmax warp of the slot
             mbar_init(&bars->o_final[s], 1);
+            mbar_init(&bars->tab_sync[s], kBM / 32);
         }
         mbar_init(&bars->mma_done, 1);
         bars->abort_flag = 0;
@@ -281,6 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool leader = elect_one();
             int kv_it = 0;
             bool ok = true;
+            // Loads issued so far (warp-uniform): each barrier has at most its last phase
+            // in flight, which the drain below waits for.  K and V load number n go to
+            // stage n % 2 and complete phase n / 2 of its barrier.
+            int nq0 = 0, nq1 = 0, nk = 0, nv = 0;
             const int nitems = items_of_cta(p);
             for (int item_it = 0; ok && item_it < nitems; ++item_it) {
                 const Item it = item_at(p, item_it);
@@ -297,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_4d(smem + L::kQ + s * L::kTile + bx * L::kBox, &tm_q, &bars->q_full[s],
                                         bx * 64, h0 + s, i0, it.b);
                     }
+                    if (s == 0) ++nq0; else ++nq1;
                 }
                 if (!ok) break;
                 if (leader && item_it + 1 < nitems) {
@@ -317,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st],
                                         bx * 64, it.g, j0, it.b);
                     }
+                    ++nk;
                     if (!(ok = warp_all(mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag)))) break;
                     if (leader) {
                         mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
@@ -324,8 +342,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st],
                                         bx * 64, it.g, j0, it.b);
                     }
+                    ++nv;
                 }
             }
+            // Drain, also after an abort: the CTA must not exit (and hand its shared
+            // memory to another CTA) while a copy into it is in flight.
+            if (nq0 > 0) mbar_drain_wait(&bars->q_full[0], (nq0 - 1) & 1);
+            if (nq1 > 0) mbar_drain_wait(&bars->q_full[1], (nq1 - 1) & 1);
+            for (int n = max(0, nk - kStages); n < nk; ++n) mbar_drain_wait(&bars->k_full[n & 1], (n >> 1) & 1);
+            for (int n = max(0, nv - kStages); n < nv; ++n) mbar_drain_wait(&bars->v_full[n & 1], (n >> 1) & 1);
         } else if (warp == 9) {
             // -------------------------------------------------------- MMA issuer
             const bool leader = elect_one();
@@ -389,10 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) umma_commit(&bars->o_final[1]);
                 }
             }
-            // Drain: wait (bounded, regardless of abort) until every MMA issued has finished.
+            // Drain: wait (bounded, regardless of abort) until every MMA issued has finished,
+            // before tensor memory is released and the CTA exits.
             if (leader) umma_commit(&bars->mma_done);
-            int dummy = 0;
-            mbar_wait(&bars->mma_done, 0, &dummy);
+            mbar_drain_wait(&bars->mma_done, 0);
         }
     } else {
         // ------------------------------------------------------------ softmax / epilogue
@@ -406,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cmax = tab_cmax(p.R);
         int tile_it = 0;
         int staged_head = -1;
+        uint32_t tab_phase = 0;
         bool ok = slot < p.nslots;
         const int nitems = items_of_cta(p);
         for (int item_it = 0; ok && item_it < nitems; ++item_it) {
@@ -418,8 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // This head's reversed distance table, NCOPY shifted copies, staged when the
             // head changes.  Loads are issued eight at a time so their L2 latencies overlap.
             if (h != staged_head) {
+            // The slot's four warps meet before the table is rewritten (all done reading
+            // the old one) and after (the new one complete).  The meeting is a bounded
+            // mbarrier wait, so a warp that has wound down after an abort cannot leave
+            // the others waiting for good.
             staged_head = h;
-            named_bar_sync(1 + slot, kBM);
+            if (!(ok = tab_meet(&bars->tab_sync[slot], tab_phase, abort_flag))) break;
             {
                 const float* wrow = p.w + static_cast<size_t>(h) * p.R;
                 for (int x0 = 0; x0 < tslot; x0 += 8 * kBM) {
@@ -438,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            named_bar_sync(1 + slot, kBM);
+            if (!(ok = tab_meet(&bars->tab_sync[slot], tab_phase, abort_flag))) break;
             }
 
             const int i = i0 + t;

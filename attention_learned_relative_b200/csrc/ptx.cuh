@@ -14,8 +14,12 @@ __device__ unsigned int g_status = 0;
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadLength = 2u;   // a device-side length or page index was out of range
 constexpr float kLn2 = 0.6931471805599453f;
-// A single wait longer than this is treated as a hang (nanoseconds).
+// A single wait longer than this is treated as a hang (nanoseconds).  Kernels read
+// the limit from g_wait_limit_ns, which the host may lower (relbias_set_wait_limit_ns)
+// to make waits run out on purpose; the waits that drain a CTA's own copies and MMAs
+// before it exits always use the fixed default.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,21 +62,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up when
-// *abort_flag is set by another thread of the CTA, or after kWaitLimitNs, in
+// *abort_flag is set by another thread of the CTA, or after g_wait_limit_ns, in
 // which case it sets the flag and the device status word.  Returns false when
 // the caller must wind down.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long limit = g_wait_limit_ns;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 *abort_flag = 1;
                 atomicOr(&g_status, kStatusTimeout);
                 return false;
             }
+        }
+    }
+}
+
+// Wait, ignoring any abort, until the phase of `bar` with the given parity completes:
+// used before a CTA exits, for copies and MMAs it issued itself, which complete
+// without help from other threads.  Bounded by the fixed kWaitLimitNs (then it sets
+// the status word and returns false).
+__device__ __forceinline__ bool mbar_drain_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, kStatusTimeout);
+            return false;
         }
     }
 }

@@ -251,29 +251,50 @@ extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int
 }
 
 namespace {
+// Host-side checks of a contiguous-cache decode call; the workspace pointer is
+// checked only when `check_ws` (the allocation-free variant supplies its own).  Sets
+// *nothing_to_do for an empty batch (after the shape checks, before any pointer
+// check).  The only CUDA calls are the device queries, made after the arguments pass.
+int decode_check_args(const void* q, const void* k_cache, const void* v_cache, const float* r, const float* w,
+                      size_t w_bstride, const void* o, const float* lse, int B, int n_ctx, int Hq, int Hkv, int d,
+                      int R, float scale, int dtype, bool check_ws, const void* workspace, bool* nothing_to_do,
+                      DeviceInfo* dev) {
+    *nothing_to_do = false;
+    int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0) {
+        *nothing_to_do = true;
+        return RELBIAS_OK;
+    }
+    if (n_ctx < 1) return fail(RELBIAS_ERR_ARG, "n_ctx (%d) must be >= 1", n_ctx);
+    if (!q || !k_cache || !v_cache || (w_bstride == 0 && !r) || !o)
+        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, r and o must not be null");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache and o must be 16-byte aligned");
+    if (!aligned4(r) || (lse && !aligned4(lse))) return fail(RELBIAS_ERR_ARG, "r and lse must be 4-byte aligned");
+    if (check_ws && (!workspace || !aligned16(workspace)))
+        return fail(RELBIAS_ERR_ARG, "workspace must be non-null and 16-byte aligned");
+    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports bf16 only");
+    if (d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports d == 128, got %d", d);
+    if (Hq / Hkv > 8) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports up to 8 query heads per key/value head");
+    if ((rc = device_info(*dev)) != RELBIAS_OK) return rc;
+    if (dev->major != 10 || dev->minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "decode needs compute capability 10.0 (sm_100a), found %d.%d",
+                    dev->major, dev->minor);
+    return RELBIAS_OK;
+}
+
 // Contiguous-cache decode.  w_bstride == 0: rank-1 tables w [Hq, R] times r [B, Hq];
 // w_bstride == Hq * R: per-sequence curves w [B, Hq, R] with coefficient 1 (r unused).
 int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* r, const float* w,
                 size_t w_bstride, void* o, float* lse, int B, int n_ctx, int Hq, int Hkv, int d, int window, int R,
                 float scale, int temp_n0, int dtype, void* workspace, size_t ws_bytes, void* stream) {
-    int rc = check_common(B, n_ctx, Hq, Hkv, d, R, scale, w);
-    if (rc != RELBIAS_OK) return rc;
-    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
-    if (B == 0) return RELBIAS_OK;
-    if (n_ctx < 1) return fail(RELBIAS_ERR_ARG, "n_ctx (%d) must be >= 1", n_ctx);
-    if (!q || !k_cache || !v_cache || (w_bstride == 0 && !r) || !o || !workspace)
-        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, r, o and workspace must not be null");
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace))
-        return fail(RELBIAS_ERR_ARG, "q, k_cache, v_cache, o and workspace must be 16-byte aligned");
-    if (!aligned4(r) || (lse && !aligned4(lse))) return fail(RELBIAS_ERR_ARG, "r and lse must be 4-byte aligned");
-    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports bf16 only");
-    if (d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports d == 128, got %d", d);
-    if (Hq / Hkv > 8) return fail(RELBIAS_ERR_UNSUPPORTED, "decode supports up to 8 query heads per key/value head");
+    bool nothing_to_do = false;
     DeviceInfo dev;
-    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
-    if (dev.major != 10 || dev.minor != 0)
-        return fail(RELBIAS_ERR_UNSUPPORTED, "decode needs compute capability 10.0 (sm_100a), found %d.%d", dev.major,
-                    dev.minor);
+    int rc = decode_check_args(q, k_cache, v_cache, r, w, w_bstride, o, lse, B, n_ctx, Hq, Hkv, d, R, scale, dtype,
+                               true, workspace, &nothing_to_do, &dev);
+    if (rc != RELBIAS_OK || nothing_to_do) return rc;
 
     DecodeParams p{};
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -512,7 +533,14 @@ extern "C" int relbias_device_status(int reset) {
     return static_cast<int>(v);
 }
 
-extern "C" int relbias_version(void) { return 400; }
+extern "C" int relbias_set_wait_limit_ns(unsigned long long ns) {
+    t_err.clear();
+    const unsigned long long v = ns == 0 ? kWaitLimitNs : ns;
+    const cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "setting the wait limit");
+}
+
+extern "C" int relbias_version(void) { return 500; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"

@@ -52,6 +52,7 @@ SIGNATURES = {
     "relbias_attn_bwd": (_I, [_VP] * 13 + [_I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
+    "relbias_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "relbias_version": (_I, []),
 }
 
@@ -380,6 +381,12 @@ def device_status(reset: bool = True) -> int:
     if rc < 0:
         _check(rc)
     return rc
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound on a single wait inside the library's kernels, in nanoseconds (0: the
+    default of 2 s).  A short bound makes waits run out on purpose (failure-path tests)."""
+    _check(lib().relbias_set_wait_limit_ns(int(ns)))
 
 
 def last_error() -> str:

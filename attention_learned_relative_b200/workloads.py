@@ -98,7 +98,7 @@ WORKLOADS = {
 }
 
 
-def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None = None):
+def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None = None, kv=None):
     """Inputs of a workload (optionally with fewer tokens or sequences), on `device`.
 
     Prefill: q [B,T,Hq,d], k/v [B,T,Hkv,d] (wl dtype), r [B,T,Hq] fp32, w [Hq,R] fp32.
@@ -108,6 +108,8 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
     seeded permutation of the pool: sequence b's logical block j is page table[b, j])
     and lens [B] int32.  The logical cache of sequence b is then k_pages[table[b]],
     not k[b]; logical_cache() returns it.
+    `kv`, if given, is a (k, v) pair drawn earlier for the same seed and shape, used
+    instead of drawing the same values again.
     """
     T = wl.T if T is None else T
     B = wl.B if B is None else B
@@ -119,8 +121,13 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, B: int | None 
     else:
         q = synth.normal((B, T, wl.Hq, wl.d), s, "q", std=wl.qk_std, dtype=dt, device=device)
         r = synth.normal((B, T, wl.Hq), s, "r", device=device)
-    k = synth.normal((B, T, wl.Hkv, wl.d), s, "k", std=wl.qk_std, dtype=dt, device=device)
-    v = synth.normal((B, T, wl.Hkv, wl.d), s, "v", dtype=dt, device=device)
+    if kv is not None:
+        k, v = kv
+        if tuple(k.shape) != (B, T, wl.Hkv, wl.d) or k.dtype != dt or v.shape != k.shape:
+            raise ValueError("kv does not match the workload's cache shape")
+    else:
+        k = synth.normal((B, T, wl.Hkv, wl.d), s, "k", std=wl.qk_std, dtype=dt, device=device)
+        v = synth.normal((B, T, wl.Hkv, wl.d), s, "v", dtype=dt, device=device)
     w = synth.normal((wl.Hq, wl.R), s, "w", std=0.5, device=device)
     x = {"q": q, "k": k, "v": v, "r": r, "w": w}
     if wl.backward:

@@ -14,6 +14,11 @@ the launching stream; with N GPUs every rank runs its own copy of the workload
 (independent units, no data-path collective: weak scaling) and the time is the max
 over ranks.  Rank 0 prints one JSON line.
 
+The default run also times every other workload (global-layer prefill at 32k and
+131k tokens, decode against a 1M-token cache in its contiguous, paged and
+shared-bank forms, and the local-layer backward pass), each in its own timed
+region with the same rules, and reports them in the same line under "per_config".
+
 --impl reference times the fp64 CPU oracle instead (the only other code path for
 this method) on a bounded sample of the same workload, on rank 0 only.
 """
@@ -51,7 +56,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token / cache length (small profiling captures only)")
-    return ap.parse_args(argv)
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only --workload (the default run also times every other workload)")
+    args = ap.parse_args(argv)
+    args.per_config = (not args.no_per_config and args.workload == DEFAULT_WORKLOAD and args.tokens is None
+                       and args.impl == "ours")
+    return args
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -175,13 +185,57 @@ def max_over_ranks(value: float, device, world: int) -> float:
 
 # ----------------------------------------------------------------------------- our arm
 
-def make_sets(wl, nsets, device):
+def input_plan(wl):
+    """Per-step input footprint, the number of independently drawn input sets the timed
+    steps rotate over (enough to exceed 3x the 126 MB L2, or one set when a single step
+    already does), and the note the JSON line carries about it."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    if wl.decode:
+        step_bytes = wl.kv_bytes()
+    else:
+        step_bytes = (2 * wl.B * wl.T * wl.Hq * wl.d + 2 * wl.B * wl.T * wl.Hkv * wl.d) * esz
+        if wl.backward:   # o and dout in, fp32 gradients out
+            step_bytes += 2 * wl.B * wl.T * wl.Hq * wl.d * esz + 4 * wl.B * wl.T * (wl.Hq + 2 * wl.Hkv) * wl.d
+    l2 = 126 * 2 ** 20
+    nsets = 1 if step_bytes > 3 * l2 else int(math.ceil(3 * l2 / step_bytes)) + 1
+    note = ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6)) if nsets > 1 \
+        else "per-step input %.0f MB > L2" % (step_bytes / 1e6)
+    return step_bytes, nsets, note
+
+
+def launches_per_step(wl) -> int:
+    """Kernels of this library one step launches."""
+    if wl.decode:
+        return 3 if wl.bank_C > 0 else 2       # (bank curves), split-KV, combine
+    return 2 if wl.backward else 1             # dq + dk/dv kernels, or the one prefill kernel
+
+
+def workload_config(wl, world, l2_note):
+    return {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+            "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
+            **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
+            **({"bias": "shared bank, C=%d functions" % wl.bank_C} if wl.bank_C > 0 else {}),
+            **({"pass": "backward (dq, dk, dv, dr, dw)"} if wl.backward else {}),
+            "parallelism": "dp%d (batch shards, no collective)" % world,
+            "l2": l2_note}
+
+
+def make_sets(wl, nsets, device, shared=None):
+    """`nsets` independently drawn input sets.  Decode workloads that draw the same
+    cache (same seed and shape) take it from `shared` instead of drawing it again."""
     import torch
     from attention_learned_relative_b200 import workloads
     from dataclasses import replace
     sets = []
     for s in range(nsets):
-        x = workloads.make_inputs(replace(wl, seed=wl.seed + 1000 * s), device=device)
+        wl_s = replace(wl, seed=wl.seed + 1000 * s)
+        kv = None
+        key = (wl_s.seed, wl.B, wl.T, wl.Hkv, wl.d, wl.dtype, wl.qk_std)
+        if wl.decode and shared is not None:
+            kv = shared.get(key)
+        x = workloads.make_inputs(wl_s, device=device, kv=kv)
+        if wl.decode and shared is not None:
+            shared[key] = (x["k"], x["v"])
         if wl.decode:
             x["o"] = torch.empty_like(x["q"])
             x["lse"] = torch.empty(wl.B, wl.Hq, dtype=torch.float32, device=device)
@@ -331,32 +385,52 @@ def cpu_baseline(wl, x, budget_s):
         "%d random (b,h,i) rows of %s (%.3g masked GFLOP, %.1f s)" % (n, wl.name, flops(rows) / 1e9, dt), dt
 
 
-def run_ours(args, wl, peaks, peaks_kind):
-    import numpy as np  # noqa: F401
-    import torch
-    import torch.distributed as dist
-    from attention_learned_relative_b200 import build, ops
+# Workloads the default run measures beside the headline one, each in its own timed
+# region, reported in the same JSON line under "per_config".
+PER_CONFIG = ["global_prefill_bf16", "global_long_prefill_bf16", "global_decode_bf16",
+              "global_decode_paged_bf16", "global_decode_bank_bf16", "local_backward_bf16"]
 
-    rank, world, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
-    build.build()  # no-op when the in-tree library is current
 
-    # Per-step footprint; rotate over enough input sets to exceed 3x the L2.
-    esz = 2 if wl.dtype == "bf16" else 4
+def roofline_of(wl, ms_step, peaks, peaks_kind):
+    """Roofline object of a workload's dominant kernel(s) at `ms_step` per step."""
+    traffic = profile_traffic(wl.name)
     if wl.decode:
-        step_bytes = wl.kv_bytes()
-    else:
-        step_bytes = (2 * wl.B * wl.T * wl.Hq * wl.d + 2 * wl.B * wl.T * wl.Hkv * wl.d) * esz
-        if wl.backward:   # o and dout in, fp32 gradients out
-            step_bytes += 2 * wl.B * wl.T * wl.Hq * wl.d * esz + 4 * wl.B * wl.T * (wl.Hq + 2 * wl.Hkv) * wl.d
-    l2 = 126 * 2 ** 20
-    nsets = 1 if step_bytes > 3 * l2 else int(math.ceil(3 * l2 / step_bytes)) + 1
-    wl, _ = rank_workload(wl, rank, world)
-    sets = make_sets(wl, nsets, dev)
+        per_step = wl.kv_bytes()
+        achieved = per_step / (ms_step * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        return per_step, {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                          "traffic": traffic, "peak_source": peaks_kind + " hbm_gbs (copy)",
+                          "kernel": ("bank_curves_kernel + " if wl.bank_C > 0 else "")
+                          + "decode_splitkv_kernel + decode_combine_kernel",
+                          "algorithmic_bytes_per_launch": per_step}
+    per_step = wl.masked_flops()
+    achieved = per_step / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    if wl.dtype != "bf16" or wl.backward:
+        # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    tensor = wl.dtype == "bf16" and not wl.backward
+    return per_step, {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                      "frac": achieved / peak, "traffic": traffic,
+                      "peak_source": (peaks_kind + " bf16_tflops (burst)") if tensor
+                      else "fp32 FMA units x max clock",
+                      "frac_of_datasheet_2250": achieved / 2250.0,
+                      "kernel": "bwd_dq_kernel + bwd_dkv_kernel" if wl.backward
+                      else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel"),
+                      "algorithmic_flops_per_launch": per_step}
+
+
+def measure(args, wl, ctx, steps_arg, e2e_on, cpu_budget, shared=None):
+    """Time one workload: W warm-up steps, then K steps between barriers and device
+    synchronisations, CUDA events on the launching stream, max over ranks.  Every rank
+    takes the same collective steps.  Returns the JSON object on rank 0, else None."""
+    import torch
+    from attention_learned_relative_b200 import ops
+
+    rank, world, dev = ctx["rank"], ctx["world"], ctx["dev"]
+    step_bytes, nsets, l2_note = input_plan(wl)
+    wl_r, _ = rank_workload(wl, rank, world)
+    sets = make_sets(wl_r, nsets, dev, shared)
     workspace = None
     if wl.backward:
         workspace = torch.empty(max(16, ops.lib().relbias_attn_bwd_workspace_size(wl.B, wl.T, wl.Hq)),
@@ -369,7 +443,7 @@ def run_ours(args, wl, peaks, peaks_kind):
         else:
             nbytes = ops.decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
-    step = step_fn(wl, ops, workspace)
+    step = step_fn(wl_r, ops, workspace)
     stream = torch.cuda.current_stream(dev)
 
     # Warm-up; then size the timed region to ~2 s unless --steps is given.
@@ -378,22 +452,24 @@ def run_ours(args, wl, peaks, peaks_kind):
         step(sets[i % nsets], stream)
     torch.cuda.synchronize()
     warm_ms = (time.perf_counter() - t0) * 1e3 / max(args.warmup, 1)
-    steps = args.steps if args.steps is not None else int(max(20, min(20000, 2000.0 / max(warm_ms, 1e-3))))
+    steps = steps_arg if steps_arg is not None else int(max(20, min(20000, 2000.0 / max(warm_ms, 1e-3))))
+    # The step count is the same on every rank (rank 0's choice).
+    steps = int(round(max_over_ranks(float(steps), dev, world))) if world > 1 else steps
     ops.device_status(reset=True)
 
     if world > 1:
-        dist.barrier()
+        torch.distributed.barrier()
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(ctx["local"]) as clocks:
         ev0.record(stream)
         for i in range(steps):
             step(sets[i % nsets], stream)
         ev1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
-        dist.barrier()
+        torch.distributed.barrier()
     ms_total = ev0.elapsed_time(ev1)
     status = ops.device_status(reset=True)
     ms_total = max_over_ranks(ms_total, dev, world)
@@ -401,7 +477,7 @@ def run_ours(args, wl, peaks, peaks_kind):
 
     # End to end through the public API: pinned host inputs -> device -> kernel -> host.
     e2e = None
-    if not args.no_e2e:
+    if e2e_on:
         x = sets[0]
         if wl.decode:
             names_in = ["q", "rs"] if wl.bank_C > 0 else ["q", "r"]
@@ -426,7 +502,7 @@ def run_ours(args, wl, peaks, peaks_kind):
         e2e_step()
         torch.cuda.synchronize()
         if world > 1:
-            dist.barrier()
+            torch.distributed.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -439,36 +515,9 @@ def run_ours(args, wl, peaks, peaks_kind):
 
     result = None
     if rank == 0:
-        traffic = profile_traffic(wl.name)
-        if wl.decode:
-            unit = "GB/s"
-            per_step = wl.kv_bytes()
-            value = per_step * world / (ms_step * 1e-3) / 1e9
-            achieved = per_step / (ms_step * 1e-3) / 1e9
-            peak = float(peaks["hbm_gbs"])
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": traffic, "peak_source": peaks_kind + " hbm_gbs (copy)",
-                    "kernel": ("bank_curves_kernel + " if wl.bank_C > 0 else "")
-                    + "decode_splitkv_kernel + decode_combine_kernel",
-                    "algorithmic_bytes_per_launch": per_step}
-        else:
-            unit = "TFLOP/s"
-            per_step = wl.masked_flops()
-            value = per_step * world / (ms_step * 1e-3) / 1e12
-            achieved = per_step / (ms_step * 1e-3) / 1e12
-            peak = float(peaks["bf16_tflops"])
-            if wl.dtype != "bf16" or wl.backward:
-                # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
-                peak = 148 * 128 * 2 * 1.965e9 / 1e12
-            tensor = wl.dtype == "bf16" and not wl.backward
-            roof = {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": traffic,
-                    "peak_source": (peaks_kind + " bf16_tflops (burst)") if tensor
-                    else "fp32 FMA units x max clock",
-                    "frac_of_datasheet_2250": achieved / 2250.0,
-                    "kernel": "bwd_dq_kernel + bwd_dkv_kernel" if wl.backward
-                    else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel"),
-                    "algorithmic_flops_per_launch": per_step}
+        per_step, roof = roofline_of(wl, ms_step, ctx["peaks"], ctx["peaks_kind"])
+        unit = roof["unit"]
+        value = per_step * world / (ms_step * 1e-3) / (1e9 if wl.decode else 1e12)
         result = {
             "metric": METRIC,
             "value": value,
@@ -482,26 +531,60 @@ def run_ours(args, wl, peaks, peaks_kind):
             "vs_baseline": None,
             "dtype": wl.dtype,
             "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
-                       "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
-                       **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
-                       **({"bias": "shared bank, C=%d functions" % wl.bank_C} if wl.bank_C > 0 else {}),
-                       **({"pass": "backward (dq, dk, dv, dr, dw)"} if wl.backward else {}),
-                       "parallelism": "dp%d (batch shards, no collective)" % world,
-                       "l2": ("%d rotating input sets (%.0f MB each) > 3x L2" % (nsets, step_bytes / 1e6))
-                       if nsets > 1 else "per-step input %.0f MB > L2" % (step_bytes / 1e6)},
+            "config": workload_config(wl, world, l2_note),
             "roofline": roof,
             "clocks": clocks.summary(),
-            "gpu_launches": steps * ((3 if wl.bank_C > 0 else 2) if wl.decode else (2 if wl.backward else 1)),
+            "gpu_launches": steps * launches_per_step(wl),
             "kernel_status": status,
         }
         if e2e is not None:
             e_val = per_step * world / (e2e["e_ms"] * 1e-3) / (1e9 if wl.decode else 1e12)
             result["e2e"] = {"value": e_val, "unit": unit, "h2d_bytes_per_step": e2e["bi"],
                              "d2h_bytes_per_step": e2e["bo"], "ms_per_step": e2e["e_ms"]}
-        if world == 1 and not args.no_cpu_baseline:
-            v, cores, desc, _ = cpu_baseline(wl, sets[0], args.cpu_seconds)
+        if world == 1 and cpu_budget is not None:
+            v, cores, desc, _ = cpu_baseline(wl, sets[0], cpu_budget)
             result["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
+    del sets, workspace
+    return result
+
+
+def run_ours(args, wl, peaks, peaks_kind):
+    import torch
+    import torch.distributed as dist
+    from attention_learned_relative_b200 import build
+    from attention_learned_relative_b200.workloads import WORKLOADS
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    build.build()  # no-op when the in-tree library is current
+    ctx = {"rank": rank, "world": world, "local": local, "dev": dev, "peaks": peaks, "peaks_kind": peaks_kind}
+
+    cpu_budget = None if args.no_cpu_baseline else args.cpu_seconds
+    result = measure(args, wl, ctx, args.steps, not args.no_e2e, cpu_budget)
+    torch.cuda.empty_cache()
+
+    if args.per_config:
+        per = {}
+        shared = {}
+        for name in PER_CONFIG:
+            pwl = WORKLOADS[name]
+            r = measure(args, pwl, ctx, args.steps, False,
+                        None if cpu_budget is None else min(cpu_budget, 4.0), shared)
+            if rank == 0:
+                per[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config",
+                                               "roofline", "clocks", "gpu_launches", "kernel_status")}
+                if "cpu_baseline" in r:
+                    per[name]["cpu_baseline"] = r["cpu_baseline"]
+            if not pwl.decode:
+                shared.clear()
+            torch.cuda.empty_cache()
+        shared.clear()
+        if rank == 0:
+            result["per_config"] = per
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -539,8 +622,7 @@ def run_reference(args, wl, steps_default=5):
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": steps,
         "warmup": warm, "ms_per_step": tot_s * 1e3 / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
-                   "window": wl.window, "R": wl.R},
+        "config": workload_config(wl, 1, input_plan(wl)[2]),
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -34,9 +34,11 @@
  *   - Return value: RELBIAS_OK (0) or a negative RELBIAS_ERR_* code.  The calls
  *     never abort the process.  relbias_last_error() describes the last failure
  *     on the calling thread.
- *   - Kernels bound every wait on an asynchronous copy or tensor-core result.  A
- *     wait that runs out records RELBIAS_STATUS_TIMEOUT in a device-side status
- *     word, the kernel winds down and returns; relbias_device_status() reads it.
+ *   - Kernels bound every wait on an asynchronous copy or tensor-core result (2 s
+ *     by default, see relbias_set_wait_limit_ns).  A wait that runs out records
+ *     RELBIAS_STATUS_TIMEOUT in a device-side status word; the kernel then waits
+ *     for the copies and MMAs it has itself issued, releases its tensor memory and
+ *     returns, leaving the context usable.  relbias_device_status() reads the word.
  */
 #ifndef RELBIAS_ATTN_H
 #define RELBIAS_ATTN_H
@@ -169,9 +171,13 @@ RELBIAS_API int relbias_attn_decode(const void* q, const void* k_cache, const vo
  *   - A call whose partials need more than that (see
  *     relbias_attn_decode_workspace_size) is rejected with RELBIAS_ERR_UNSUPPORTED
  *     and launches nothing.
- *   - The first call on a device looks up the scratch's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before
- *     any stream capture.
+ *   - Argument errors are reported exactly as relbias_attn_decode reports them,
+ *     before anything else happens.
+ *   - Every call looks up the scratch's device address (cudaGetSymbolAddress, a
+ *     host-side query that allocates nothing) in the device and context current
+ *     at the call, so the address stays right after cudaDeviceReset or a context
+ *     switch.  The first call on a device may load the library's device image
+ *     there; make that first call before any stream capture.
  *   - All calls on a device share the one scratch array, which keeps the last
  *     call's contents (every value a call reads it writes first).  Calls that
  *     overlap on the GPU -- on different streams without ordering between them --
@@ -298,6 +304,16 @@ RELBIAS_API const char* relbias_last_error(void);
  * accumulated since the last reset (RELBIAS_STATUS_*) and, if reset != 0,
  * clears them.  Returns a negative RELBIAS_ERR_CUDA on a CUDA failure. */
 RELBIAS_API int relbias_device_status(int reset);
+
+/* Sets the bound on a single wait inside this library's kernels on the current
+ * device, in nanoseconds (0 restores the default of 2 s).  Kernels launched after
+ * the call use it.  A short bound makes waits run out on purpose, which tests the
+ * failure path: the kernel records RELBIAS_STATUS_TIMEOUT, winds down and returns,
+ * and its outputs are then undefined.  The waits by which a kernel drains its own
+ * copies and MMAs before exiting always keep the 2 s bound.  The pages have no
+ * counterpart; this is a property of the library.  Synchronous with respect to the
+ * host (a cudaMemcpyToSymbol); returns RELBIAS_OK or RELBIAS_ERR_CUDA. */
+RELBIAS_API int relbias_set_wait_limit_ns(unsigned long long ns);
 
 /* Library version as major*10000 + minor*100 + patch. */
 RELBIAS_API int relbias_version(void);

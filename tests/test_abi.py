@@ -270,3 +270,35 @@ def test_bwd_empty_and_workspace_size(lib):
     assert _bwd(lib, T=0) == ops.RELBIAS_OK
     assert ops.lib().relbias_attn_bwd_workspace_size(2, 100, 8) == 2 * 100 * 8 * 4
     assert ops.lib().relbias_attn_bwd_workspace_size(0, 100, 8) == 16
+
+
+def _dec_noalloc(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=2, N=100, Hq=8, Hkv=1, d=128,
+             window=0, R=16, scale=0.1, temp_n0=0, dtype=ops.RELBIAS_BF16)
+    a.update(kw)
+    return lib.relbias_attn_decode_noalloc(a["q"], a["k"], a["v"], a["r"], a["w"], a["o"], a["lse"], a["B"],
+                                           a["N"], a["Hq"], a["Hkv"], a["d"], a["window"], a["R"], a["scale"],
+                                           a["temp_n0"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(r=None), dict(o=FAKE + 8), dict(k=FAKE + 2), dict(lse=FAKE + 1), dict(N=0),
+    dict(Hq=12, Hkv=8), dict(scale=0.0), dict(R=-1), dict(w=None), dict(dtype=9),
+    dict(dtype=ops.RELBIAS_FP32), dict(d=64), dict(Hq=16, Hkv=1),
+    dict(),   # valid arguments: both then fail alike at the device query on a host without a GPU
+])
+def test_noalloc_reports_argument_errors_like_the_regular_decode(lib, kw):
+    """The allocation-free decode checks its arguments before it looks up its static
+    scratch, and reports them with the regular entry point's code and message."""
+    rc_ref = _dec(lib, **kw)
+    msg_ref = ops.last_error()
+    rc = _dec_noalloc(lib, **kw)
+    assert rc == rc_ref
+    assert ops.last_error() == msg_ref
+    if kw:
+        assert rc in (ops.RELBIAS_ERR_ARG, ops.RELBIAS_ERR_UNSUPPORTED)
+
+
+def test_noalloc_empty_batch(lib):
+    assert _dec_noalloc(lib, B=0) == ops.RELBIAS_OK
+    assert _dec_noalloc(lib, B=0, q=None, o=None) == ops.RELBIAS_OK

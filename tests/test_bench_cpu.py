@@ -49,17 +49,56 @@ def test_decode_bytes_are_the_attended_cache_rows():
     assert win.kv_bytes() == 2 * wl.B * wl.Hkv * 512 * wl.d * 2
 
 
-def test_committed_ncu_summaries_describe_the_current_kernels():
+def test_committed_ncu_summaries_carry_their_source_digest(monkeypatch):
     """Every ncu summary under profiles/ names the digest of the CUDA sources it was taken
-    on; it must be the digest of the sources in the tree."""
+    on, and most give DRAM bytes per launch.  The benchmark uses those bytes as the
+    roofline's `traffic` only while the digest matches the sources in the tree; a stale
+    summary, or one without the figure, gives null."""
     import re
     prof = os.path.join(ROOT, "profiles")
     found = 0
     for name in sorted(os.listdir(prof)):
         if not name.startswith("ncu_"):
             continue
-        m = re.search(r"source_sha256:\s*([0-9a-f]+)", open(os.path.join(prof, name)).read())
+        text = open(os.path.join(prof, name)).read()
+        m = re.search(r"source_sha256:\s*([0-9a-f]{16})", text)
         assert m, name
-        assert m.group(1) == bench.source_digest(), name
+        has_bytes = re.search(r"dram_bytes_per_launch:\s*[0-9.eE+]+", text) is not None
+        workload = name[len("ncu_"):-len(".md")]
+        assert workload in WORKLOADS, name
+        current = m.group(1) == bench.source_digest() and has_bytes
+        assert (bench.profile_traffic(workload) is not None) == current, name
+        monkeypatch.setattr(bench, "source_digest", lambda: "0" * 16)
+        assert bench.profile_traffic(workload) is None, name
+        monkeypatch.undo()
         found += 1
     assert found >= 3
+
+
+def test_default_run_times_every_workload_in_one_line():
+    """The default invocation (the driver's) measures the headline workload and every
+    workload in PER_CONFIG; any other --workload times only itself."""
+    a = bench.parse_args([])
+    assert a.per_config and a.workload == bench.DEFAULT_WORKLOAD
+    assert not bench.parse_args(["--workload", "global_prefill_bf16"]).per_config
+    assert not bench.parse_args(["--no-per-config"]).per_config
+    assert not bench.parse_args(["--tokens", "1024"]).per_config
+    assert not bench.parse_args(["--impl", "reference"]).per_config
+    names = set(bench.PER_CONFIG)
+    assert names <= set(WORKLOADS) and bench.DEFAULT_WORKLOAD not in names
+    for want in ("global_prefill_bf16", "global_long_prefill_bf16", "global_decode_bf16",
+                 "global_decode_paged_bf16", "global_decode_bank_bf16"):
+        assert want in names
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_input_plan_exceeds_l2(name):
+    """Steps rotate over enough input sets that their footprint exceeds 3x the L2, or one
+    step alone exceeds it."""
+    wl = WORKLOADS[name]
+    step_bytes, nsets, note = bench.input_plan(wl)
+    l2 = 126 * 2 ** 20
+    assert step_bytes * nsets > 3 * l2 or (nsets == 1 and step_bytes > 3 * l2)
+    cfg = bench.workload_config(wl, 1, note)
+    assert cfg["workload"] == name and cfg["l2"] == note and cfg["global_batch"] == wl.B
+    assert bench.launches_per_step(wl) >= 1

@@ -130,3 +130,20 @@ def test_decode_workload_sampled():
                                      x["w"][heads].cpu().reshape(G, 1, wl.R), k_sl, v_sl, req, G, wl.window, wl.R,
                                      wl.scale)
         assert_bf16_close(o[b, heads], o_ref, lse[b, heads], lse_ref, "decode workload (b=%d, g=%d)" % (b, g))
+
+
+def test_decode_small_group_reads_only_its_own_features():
+    """Group size 4 (fewer query heads than the kernel's 8 head columns): the padding
+    columns must not read r.  r sits at the very end of a buffer whose next elements
+    are NaN; reading them would still leave O finite, so the check here is that the
+    result equals the same call with r in a buffer of its own, bit for bit."""
+    B, N, Hq, Hkv, d, R = 3, 700, 8, 2, 128, 256
+    x = _inputs(B, N, Hq, Hkv, d, R, seed=4242)
+    o_ref, lse_ref = _run(x, 0, R, 0.1)
+    buf = torch.full((B * Hq + 64,), float("nan"), dtype=torch.float32, device="cuda")
+    buf[:B * Hq] = x["r"].reshape(-1)
+    x_tail = dict(x, r=buf[:B * Hq].view(B, Hq))
+    o, lse = _run(x_tail, 0, R, 0.1)
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    o_or, lse_or = O.attn_decode(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), 0, R, 0.1)
+    assert_bf16_close(o, o_or, lse, lse_or, "decode group 4")
