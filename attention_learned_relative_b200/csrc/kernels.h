@@ -30,8 +30,17 @@ struct PrefillParams {
     float inv_scale;         // 1 / scale
     int temp_n0;             // > 1: logits of a row seeing n > temp_n0 keys are scaled by ln n / ln temp_n0
     float inv_log_n0;        // 1 / ln(temp_n0)
+    // Shared-bank form (curves != nullptr): each row's bias curve, padded rows of
+    // curve_stride floats written by launch_bank_rows; r and w are then unused.
+    const float* curves;
+    int curve_stride;
 };
 int prefill_bf16_table_copies(int d, int R);   // 0 if R does not fit shared memory
+// Shared-bank curves of every prefill row: [B, T, Hq] rows of prefill_bank_curve_stride(R)
+// floats (see bank_rows_kernel in prefill_sm100.cu).
+int prefill_bank_curve_stride(int R);
+cudaError_t launch_bank_rows(const float* rs, const float* proj, float* curves, int B, int T, int Hq, int q_off, int C,
+                             int proj_heads, int R, cudaStream_t stream);
 int prefill_bf16_smem_bytes(int d, int R);
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream);

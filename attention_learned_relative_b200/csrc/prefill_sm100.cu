@@ -233,6 +233,34 @@ __device__ __forceinline__ void add_bias(float (&s)[kBN], const float* run, floa
     }
 }
 
+// s[c] += rs * curve[delta0 + t - c] for the 128 columns, from this row's curve of
+// the shared bank in global memory (the bank form: the row has its own curve).  `row`
+// points at distance 0 of the row's padded curve and dlo = delta0 + t - 127 is the
+// distance of column 127; the padding makes row + dlo a 32-byte boundary.  Eight
+// distances per 32-byte load, columns descending; loads that reach no distance in
+// [0, R) are skipped (zeros).
+__device__ __forceinline__ void add_bias_curves(float (&s)[kBN], const float* row, int dlo, int R, float rs) {
+    const uint64_t rs2 = f2_pack(rs, rs);
+#pragma unroll
+    for (int v = 0; v < kBN / 8; ++v) {
+        const int d0 = dlo + 8 * v;   // distances d0 .. d0+7 <-> columns 127-8v .. 120-8v
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (d0 + 7 >= 0 && d0 < R) {
+            a = __ldg(reinterpret_cast<const float4*>(row + d0));
+            b = __ldg(reinterpret_cast<const float4*>(row + d0 + 4));
+        }
+        const float w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int c = kBN - 2 - 8 * v - 2 * m;   // columns c, c+1 <-> distances d0+1+2m, d0+2m
+            const uint64_t r2 = f2_fma(rs2, f2_pack(w[2 * m + 1], w[2 * m]), f2_pack(s[c], s[c + 1]));
+            f2_unpack(r2, s[c], s[c + 1]);
+        }
+    }
+}
+
+// NCOPY == 0: the shared-bank form, with each row's bias curve read from global
+// memory (no staged table).
 template <int D, int NCOPY>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -443,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // This head's reversed distance table, NCOPY shifted copies, staged when the
             // head changes.  Loads are issued eight at a time so their L2 latencies overlap.
-            if (h != staged_head) {
+            if (NCOPY > 0 && h != staged_head) {
             // The slot's four warps meet before the table is rewritten (all done reading
             // the old one) and after (the new one complete).  The meeting is a bounded
             // mbarrier wait, so a warp that has wound down after an abort cannot leave
@@ -473,8 +501,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             const int i = i0 + t;
             const bool row_ok = i < p.T;
-            const float rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale
-                                    : 0.0f;
+            // Bias coefficient, in units of the unscaled logit: r_i / scale (rank-1 form), or
+            // 1 / scale for the bank form, whose curve holds the whole bias.
+            float rs = 0.0f;
+            const float* curve_row = nullptr;
+            if constexpr (NCOPY == 0) {
+                rs = row_ok ? p.inv_scale : 0.0f;
+                curve_row = p.curves +
+                            (static_cast<size_t>(it.b) * p.T + (row_ok ? i : 0)) * p.Hq * p.curve_stride +
+                            static_cast<size_t>(h) * p.curve_stride + (7 - ((p.q_off + i) & 7));
+            } else {
+                rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale : 0.0f;
+            }
             float m_used = -INFINITY;   // running max, log2 units
             uint64_t l2 = 0;            // running sum, two partial lanes (0.0f, 0.0f)
             // Logit scale of this row, log2 units, with the context-length temperature:
@@ -507,7 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // of the unscaled logit; the table is zero outside [0, R)).
                     const int base = cmax - delta0 - t;
                     const int cp = base & (NCOPY - 1);
-                    add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
+                    if constexpr (NCOPY == 0) {
+                        if (row_ok) {
+                            add_bias_curves(s, curve_row, delta0 + t - (kBN - 1), p.R, rs);
+                            // The next tile's run (128 distances further) into L2 meanwhile.
+                            const int dn = delta0 + t + 1;   // its first distance
+                            if (tt + 1 < ntiles && dn < p.R)
+                                for (int k = 0; k < kBN; k += 32) prefetch_l2(curve_row + dn + k);
+                        }
+                    } else {
+                        add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
+                    }
                 }
                 if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
                     // Key c is visible to row t iff lo <= c <= hi.  A 32-column chunk the
@@ -642,6 +690,52 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
 
 }  // namespace
 
+// Curves of the shared bank for every (sequence, row, head) of a prefill, into the
+// padded layout the kernel's curve variant reads ("Thinking Machines dropped RoPE",
+// recipe step 2: the token's coefficients times the bank's functions):
+//   out[row * S + pad + dist] = sum_c rs[row, c] * proj[hp, c, dist]   for dist in [0, R)
+// and zeros elsewhere in the row, with row = (b * T + i) * Hq + h, hp = 0 or h, and
+// pad = 7 - (position & 7): a prefill thread's run of 128 distances for one key tile
+// then starts on a 32-byte boundary.  A block covers 16 rows of one (sequence, head)
+// and 256 distances; each thread one distance for all 16 rows, so a function value is
+// read once and used 16 times.
+constexpr int kCurveRows = 16;
+constexpr int kCurveCols = 256;
+
+__global__ void __launch_bounds__(kCurveCols) bank_rows_kernel(const float* __restrict__ rs,
+                                                               const float* __restrict__ proj,
+                                                               float* __restrict__ out, int B, int T, int Hq,
+                                                               int q_off, int C, int proj_heads, int R, int S) {
+    __shared__ float coef[kCurveRows][kMaxBankC];
+    const int iblocks = (T + kCurveRows - 1) / kCurveRows;
+    const int rb = blockIdx.x;                        // (b, h, row block)
+    const int ib = rb % iblocks;
+    const int bh = rb / iblocks;
+    const int h = bh % Hq, b = bh / Hq;
+    const int i_base = ib * kCurveRows;
+    for (int x = threadIdx.x; x < kCurveRows * C; x += blockDim.x) {
+        const int k = x / C, c = x % C;
+        const int i = i_base + k;
+        coef[k][c] = i < T ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
+    }
+    __syncthreads();
+    const int dist = static_cast<int>(blockIdx.y) * kCurveCols + static_cast<int>(threadIdx.x) - 8;
+    const bool inside = dist >= 0 && dist < R;
+    float pc[kMaxBankC];
+    const float* bank = proj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
+#pragma unroll
+    for (int c = 0; c < kMaxBankC; ++c) pc[c] = (c < C && inside) ? __ldg(bank + static_cast<size_t>(c) * R + dist) : 0.0f;
+    for (int k = 0; k < kCurveRows; ++k) {
+        const int i = i_base + k;
+        if (i >= T) break;
+        float acc = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kMaxBankC; ++c) acc = fmaf(coef[k][c], pc[c], acc);   // pc[c] = 0 for c >= C
+        const int x = dist + (7 - ((q_off + i) & 7));
+        if (x >= 0 && x < S) out[((static_cast<size_t>(b) * T + i) * Hq + h) * S + x] = inside ? acc : 0.0f;
+    }
+}
+
 int prefill_bf16_table_copies(int d, int R) {
     for (int nc = 4; nc >= 1; nc >>= 1)
         if (smem_bytes_for(d, R, nc) <= kMaxDynSmem) return nc;
@@ -657,8 +751,27 @@ int prefill_bf16_smem_bytes(int d, int R) {
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
+int prefill_bank_curve_stride(int R) { return ((R + 14) + 7) / 8 * 8; }
+
+cudaError_t launch_bank_rows(const float* rs, const float* proj, float* curves, int B, int T, int Hq, int q_off, int C,
+                             int proj_heads, int R, cudaStream_t stream) {
+    if (B < 1 || T < 1 || R < 1) return cudaSuccess;
+    const int S = prefill_bank_curve_stride(R);
+    const long long rblocks = static_cast<long long>(B) * Hq * ((T + kCurveRows - 1) / kCurveRows);
+    if (rblocks > INT32_MAX) return cudaErrorInvalidValue;
+    dim3 grid(static_cast<unsigned>(rblocks), (S + 8 + kCurveCols - 1) / kCurveCols);
+    bank_rows_kernel<<<grid, kCurveCols, 0, stream>>>(rs, proj, curves, B, T, Hq, q_off, C, proj_heads, R, S);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream) {
+    if (p.curves != nullptr) {
+        // The bank form: no staged table (shared memory as for R = 0).
+        const int smem = std::max(smem_bytes_for(d, 0, 0), 120 * 1024);
+        if (d == 128) return launch_variant<128, 0>(tq, tk, tv, p, smem, grid, stream);
+        return launch_variant<64, 0>(tq, tk, tv, p, smem, grid, stream);
+    }
     const int nc = prefill_bf16_table_copies(d, p.R);
     const int smem = prefill_bf16_smem_bytes(d, p.R);
     if (nc == 0 || smem < 0) return cudaErrorInvalidValue;

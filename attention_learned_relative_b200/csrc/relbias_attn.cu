@@ -113,6 +113,12 @@ int check_common(int B, int T, int Hq, int Hkv, int d, int R, float scale, const
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Bytes of the bf16 bank prefill's curve workspace: [B, T, Hq] padded rows.
+size_t bank_prefill_curve_bytes(int B, int T, int Hq, int R) {
+    const size_t b = static_cast<size_t>(B) * T * Hq * prefill_bank_curve_stride(R) * sizeof(float);
+    return (b + 255) / 256 * 256;
+}
+
 }  // namespace
 }  // namespace relbias
 
@@ -126,7 +132,8 @@ namespace {
 // coefficients, w [proj_heads, C, R] functions), fp32 only.
 int fwd_impl(const void* q, const void* k, const void* v, const float* r, const float* w, void* o, float* lse, int B,
              int T, int q_off, int kv_T, int Hq, int Hkv, int d, int window, int R, float scale, int temp_n0,
-             int dtype, void* stream, int C = 0, int proj_heads = 0) {
+             int dtype, void* stream, int C = 0, int proj_heads = 0, void* workspace = nullptr,
+             size_t ws_bytes = 0) {
     int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
     if (rc != RELBIAS_OK) return rc;
     if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
@@ -149,12 +156,18 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* r, const 
         return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "fp32 prefill launch");
     }
 
-    if (C > 0)
-        return fail(RELBIAS_ERR_UNSUPPORTED,
-                    "the shared-bank bias runs on the fp32 prefill path only (bf16 prefill takes the rank-1 form)");
     if (d != 64 && d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill supports d in {64, 128}, got %d", d);
     if (R > 2048 || prefill_bf16_table_copies(d, R) == 0)
         return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
+    size_t curve_bytes = 0;
+    if (C > 0 && R > 0) {
+        curve_bytes = bank_prefill_curve_bytes(B, T, Hq, R);
+        if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 31u) != 0)
+            return fail(RELBIAS_ERR_ARG, "the bf16 shared-bank prefill needs a 32-byte aligned workspace");
+        if (ws_bytes < curve_bytes)
+            return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes of bank curves",
+                        ws_bytes, curve_bytes);
+    }
     DeviceInfo dev;
     if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
     if (dev.major != 10 || dev.minor != 0)
@@ -195,6 +208,13 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* r, const 
     p.inv_scale = 1.0f / scale;
     p.temp_n0 = temp_n0 > 1 ? temp_n0 : 0;
     p.inv_log_n0 = temp_n0 > 1 ? static_cast<float>(1.0 / std::log(static_cast<double>(temp_n0))) : 0.0f;
+    if (C > 0 && R > 0) {
+        // Shared bank: each row's curve sum_c rs[c] * proj[c, dist] first, into the workspace.
+        cudaError_t e = launch_bank_rows(r, w, static_cast<float*>(workspace), B, T, Hq, q_off, C, proj_heads, R, st);
+        if (e != cudaSuccess) return cuda_fail(e, "bank curve launch");
+        p.curves = static_cast<const float*>(workspace);
+        p.curve_stride = prefill_bank_curve_stride(R);
+    }
     const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
     cudaError_t e = launch_prefill_bf16_sm100(tq, tk, tv, p, d, grid, st);
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "bf16 prefill launch");
@@ -232,14 +252,21 @@ size_t bank_curve_bytes(int B, int Hq, int R) {
 }  // namespace
 }  // namespace relbias
 
+extern "C" size_t relbias_attn_fwd_bank_workspace_size(int B, int T, int Hq, int R, int dtype) {
+    if (B < 0 || T < 0 || Hq < 1 || R < 0) return 0;
+    if (dtype != RELBIAS_BF16 || R == 0) return 0;
+    return bank_prefill_curve_bytes(B, T, Hq, R);
+}
+
 extern "C" int relbias_attn_fwd_bank(const void* q, const void* k, const void* v, const float* rs, const float* proj,
                                      void* o, float* lse, int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
-                                     int window, int R, float scale, int temp_n0, int dtype, void* stream) {
+                                     int window, int R, float scale, int temp_n0, int dtype, void* workspace,
+                                     size_t ws_bytes, void* stream) {
     t_err.clear();
     const int rc = check_bank(C, proj_heads, Hq);
     if (rc != RELBIAS_OK) return rc;
     return fwd_impl(q, k, v, rs, proj, o, lse, B, T, 0, T, Hq, Hkv, d, window, R, scale, temp_n0, dtype, stream, C,
-                    proj_heads);
+                    proj_heads, workspace, ws_bytes);
 }
 
 extern "C" size_t relbias_attn_decode_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d, int window) {
@@ -540,7 +567,7 @@ extern "C" int relbias_set_wait_limit_ns(unsigned long long ns) {
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "setting the wait limit");
 }
 
-extern "C" int relbias_version(void) { return 500; }
+extern "C" int relbias_version(void) { return 600; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"

@@ -43,8 +43,9 @@ SIGNATURES = {
     "relbias_attn_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode_paged": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
                                        _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
+    "relbias_attn_fwd_bank_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "relbias_attn_fwd_bank": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
-                                   _I, _VP]),
+                                   _I, _VP, _SZ, _VP]),
     "relbias_attn_decode_bank_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode_bank": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                       _I, _VP, _SZ, _VP]),
@@ -278,27 +279,40 @@ def _bank_shape(proj, C_from_rs: int, Hq: int, R: int) -> int:
     return int(proj.shape[0])
 
 
+def fwd_bank_workspace_size(B: int, T: int, Hq: int, R: int, dtype: int) -> int:
+    """Bytes of scratch attn_fwd_bank needs (0: none, for the fp32 path)."""
+    return int(lib().relbias_attn_fwd_bank_workspace_size(B, T, Hq, R, dtype))
+
+
 def attn_fwd_bank(q, k, v, rs, proj, window: int, R: int, scale: float | None = None, out=None, lse=None,
-                  stream=None, temp_n0: int = 0):
+                  stream=None, temp_n0: int = 0, workspace=None):
     """Prefill with the shared-bank bias sum_c rs[b,i,h,c] * proj[h or 0, c, i-j].
-    q [B,T,Hq,d], k/v [B,T,Hkv,d] fp32 (the bank form runs on the fp32 path),
-    rs [B,T,Hq,C] fp32, proj [1 or Hq, C, R] fp32.  Returns o [B,T,Hq,d]."""
+    q [B,T,Hq,d], k/v [B,T,Hkv,d] (bf16 or fp32), rs [B,T,Hq,C] fp32,
+    proj [1 or Hq, C, R] fp32.  Returns o [B,T,Hq,d].  The bf16 path writes every
+    row's curve into `workspace` (a byte tensor of at least fwd_bank_workspace_size
+    bytes; allocated if None) before the tensor-core kernel reads it."""
     _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
     _need(rs.dim() == 4 and rs.shape[:3] == (B, T, Hq) and rs.dtype == torch.float32, "rs must be fp32 [B,T,Hq,C]")
     C = int(rs.shape[3])
     proj_heads = _bank_shape(proj, C, Hq, R)
-    for t in (q, k, v, rs, proj, out, lse):
+    for t in (q, k, v, rs, proj, out, lse, workspace):
         _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
     if out is None:
         out = torch.empty_like(q)
     _need(lse is None or (lse.shape == (B, Hq, T) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq,T]")
+    code = _dtype_code(q)
+    need = fwd_bank_workspace_size(B, T, Hq, R, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     rc = lib().relbias_attn_fwd_bank(_ptr(q), _ptr(k), _ptr(v), _ptr(rs), _ptr(proj), _ptr(out), _ptr(lse),
                                      B, T, Hq, Hkv, d, C, proj_heads, int(window), int(R), float(scale),
-                                     int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
+                                     int(temp_n0), code, _ptr(workspace), ws_bytes,
+                                     _stream_handle(stream, q.device))
     _check(rc)
     return out
 

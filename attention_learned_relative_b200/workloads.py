@@ -91,6 +91,10 @@ WORKLOADS = {
         # distance shared by all heads, 16 coefficients per (token, head).
         Workload("global_decode_bank_bf16", B=8, T=1048576, Hq=32, Hkv=4, d=128, window=0,
                  R=1024, seed=4, dtype="bf16", decode=True, bank_C=16),
+        # The local-layer prefill with the essay's shared bank: 16 functions of distance
+        # shared by all heads, 16 coefficients per (token, head).
+        Workload("local_prefill_bank_bf16", B=2, T=8192, Hq=32, Hkv=4, d=128, window=512, R=512,
+                 seed=1, dtype="bf16", bank_C=16),
         # The backward pass of the local-layer prefill (the pages train the model).
         Workload("local_backward_bf16", B=2, T=8192, Hq=32, Hkv=4, d=128, window=512, R=512,
                  seed=1, dtype="bf16", backward=True),

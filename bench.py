@@ -207,6 +207,8 @@ def launches_per_step(wl) -> int:
     """Kernels of this library one step launches."""
     if wl.decode:
         return 3 if wl.bank_C > 0 else 2       # (bank curves), split-KV, combine
+    if wl.bank_C > 0:
+        return 2                               # bank curves, prefill
     return 2 if wl.backward else 1             # dq + dk/dv kernels, or the one prefill kernel
 
 
@@ -269,6 +271,10 @@ def step_fn(wl, ops, workspace):
         def step(x, stream):
             ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
                             lse=x["lse"], workspace=workspace, stream=stream)
+    elif wl.bank_C > 0:
+        def step(x, stream):
+            ops.attn_fwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], wl.window, wl.R, wl.scale, out=x["o"],
+                              lse=x["lse"], stream=stream, workspace=workspace)
     elif wl.backward:
         def step(x, stream):
             ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], x["o"], x["lse"], x["dout"], wl.window, wl.R,
@@ -353,7 +359,12 @@ def cpu_baseline(wl, x, budget_s):
 
     k_cpu = x["k"].cpu()
     v_cpu = x["v"].cpu()
-    proj = x["w"].cpu().reshape(wl.Hq, 1, wl.R)
+    if wl.bank_C > 0:
+        proj = x["proj"].cpu()                       # [1, C, R], shared by the heads
+        coef = x["rs"]                               # [B, T, Hq, C]
+    else:
+        proj = x["w"].cpu().reshape(wl.Hq, 1, wl.R)
+        coef = x["r"][..., None]                     # [B, T, Hq, 1]
 
     def draw(n):
         b = torch.randint(0, wl.B, (n,), generator=g)
@@ -361,9 +372,9 @@ def cpu_baseline(wl, x, budget_s):
         i = torch.randint(0, wl.T, (n,), generator=g)
         idx = [t.to(x["q"].device) for t in (b, i, h)]
         q = x["q"][idx[0], idx[1], idx[2]].float().cpu()
-        r = x["r"][idx[0], idx[1], idx[2]].cpu()
+        r = coef[idx[0], idx[1], idx[2]].cpu()
         rows = torch.stack([b, h, i], 1).numpy().astype(np.int64)
-        return rows, q, r.reshape(-1, 1)
+        return rows, q, r.reshape(n, -1)
 
     def flops(rows):
         i = rows[:, 2]
@@ -387,7 +398,7 @@ def cpu_baseline(wl, x, budget_s):
 
 # Workloads the default run measures beside the headline one, each in its own timed
 # region, reported in the same JSON line under "per_config".
-PER_CONFIG = ["global_prefill_bf16", "global_long_prefill_bf16", "global_decode_bf16",
+PER_CONFIG = ["local_prefill_bank_bf16", "global_prefill_bf16", "global_long_prefill_bf16", "global_decode_bf16",
               "global_decode_paged_bf16", "global_decode_bank_bf16", "local_backward_bf16"]
 
 
@@ -416,7 +427,8 @@ def roofline_of(wl, ms_step, peaks, peaks_kind):
                       else "fp32 FMA units x max clock",
                       "frac_of_datasheet_2250": achieved / 2250.0,
                       "kernel": "bwd_dq_kernel + bwd_dkv_kernel" if wl.backward
-                      else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel"),
+                      else ("bank_rows_kernel + prefill_bf16_sm100_kernel" if wl.bank_C > 0 and wl.dtype == "bf16"
+                            else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel")),
                       "algorithmic_flops_per_launch": per_step}
 
 
@@ -435,6 +447,10 @@ def measure(args, wl, ctx, steps_arg, e2e_on, cpu_budget, shared=None):
     if wl.backward:
         workspace = torch.empty(max(16, ops.lib().relbias_attn_bwd_workspace_size(wl.B, wl.T, wl.Hq)),
                                 dtype=torch.uint8, device=dev)
+    if wl.bank_C > 0 and not wl.decode:
+        nbytes = ops.fwd_bank_workspace_size(wl.B, wl.T, wl.Hq, wl.R,
+                                             ops.RELBIAS_BF16 if wl.dtype == "bf16" else ops.RELBIAS_FP32)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     if wl.decode:
         if wl.page_size > 0:
             nbytes = ops.decode_paged_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.window)
@@ -483,6 +499,8 @@ def measure(args, wl, ctx, steps_arg, e2e_on, cpu_budget, shared=None):
             names_in = ["q", "rs"] if wl.bank_C > 0 else ["q", "r"]
         elif wl.backward:
             names_in = ["q", "k", "v", "r", "w", "o", "lse", "dout"]
+        elif wl.bank_C > 0:
+            names_in = ["q", "k", "v", "rs", "proj"]
         else:
             names_in = ["q", "k", "v", "r", "w"]
         host_in = {n: x[n].cpu().pin_memory() for n in names_in}

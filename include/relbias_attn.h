@@ -237,10 +237,15 @@ RELBIAS_API int relbias_attn_decode_paged(const void* q, const void* k_pages, co
  * head, proj_heads = Hq).  The rank-1 form of relbias_attn_fwd is the case
  * C = 1, proj_heads = Hq.  1 <= C <= 16.
  *
- * relbias_attn_fwd_bank: prefill, RELBIAS_FP32 only (the bf16 tensor-core
- * kernel takes the rank-1 form and returns RELBIAS_ERR_UNSUPPORTED here).
+ * relbias_attn_fwd_bank: prefill.
  *   rs   [B, T, Hq, C]          fp32
  *   proj [proj_heads, C, R]     fp32   (may be NULL if R == 0)
+ *   workspace, ws_bytes: RELBIAS_BF16 only (NULL and 0 for RELBIAS_FP32): caller-owned
+ *        device scratch of at least relbias_attn_fwd_bank_workspace_size(...) bytes,
+ *        32-byte aligned.  The bf16 path first writes every row's curve
+ *        sum_c rs[b,i,h,c] * proj[h', c, :] there (one padded fp32 row of R + 14..21
+ *        floats per (b, i, h)), then the tensor-core kernel reads each row's curve in
+ *        place of the rank-1 r * w; the fp32 path evaluates the sum per key itself.
  *   other arguments as for relbias_attn_fwd.
  *
  * relbias_attn_decode_bank: decode as relbias_attn_decode, with
@@ -251,12 +256,14 @@ RELBIAS_API int relbias_attn_decode_paged(const void* q, const void* k_pages, co
  * read those curves.  ws_bytes must be at least
  * relbias_attn_decode_bank_workspace_size(...).
  */
+RELBIAS_API size_t relbias_attn_fwd_bank_workspace_size(int B, int T, int Hq, int R, int dtype);
+
 RELBIAS_API int relbias_attn_fwd_bank(const void* q, const void* k, const void* v,
-                     const float* rs, const float* proj,
-                     void* o, float* lse,
-                     int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
-                     int window, int R, float scale, int temp_n0,
-                     int dtype, void* stream);
+                        const float* rs, const float* proj,
+                        void* o, float* lse,
+                        int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
+                        int window, int R, float scale, int temp_n0,
+                        int dtype, void* workspace, size_t ws_bytes, void* stream);
 RELBIAS_API size_t relbias_attn_decode_bank_workspace_size(int B, int Hq, int Hkv, int n_ctx, int d,
                                           int window, int R);
 RELBIAS_API int relbias_attn_decode_bank(const void* q, const void* k_cache, const void* v_cache,

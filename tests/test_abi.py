@@ -48,7 +48,16 @@ def test_binding_argument_counts_match_header():
 
 
 def test_version(lib):
-    assert ops.version() >= 400
+    assert ops.version() >= 600
+
+
+def test_fwd_bank_workspace_size(lib):
+    # bf16: [B, T, Hq] rows of R + 14 floats rounded up to 8, rounded up to 256 bytes; fp32: none.
+    stride = (16 + 14 + 7) // 8 * 8
+    want = (2 * 10 * 4 * stride * 4 + 255) // 256 * 256
+    assert ops.fwd_bank_workspace_size(2, 10, 4, 16, ops.RELBIAS_BF16) == want
+    assert ops.fwd_bank_workspace_size(2, 10, 4, 16, ops.RELBIAS_FP32) == 0
+    assert ops.fwd_bank_workspace_size(2, 10, 4, 0, ops.RELBIAS_BF16) == 0
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
@@ -193,11 +202,11 @@ def test_chunk_empty_is_a_no_op(lib):
 
 def _fwd_bank(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, rs=FAKE, proj=FAKE, o=FAKE, lse=None, B=1, T=8, Hq=4, Hkv=2, d=64, C=16,
-             proj_heads=1, window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_FP32)
+             proj_heads=1, window=0, R=16, scale=0.125, temp_n0=0, dtype=ops.RELBIAS_FP32, ws=None, ws_bytes=0)
     a.update(kw)
     return lib.relbias_attn_fwd_bank(a["q"], a["k"], a["v"], a["rs"], a["proj"], a["o"], a["lse"], a["B"], a["T"],
                                      a["Hq"], a["Hkv"], a["d"], a["C"], a["proj_heads"], a["window"], a["R"],
-                                     a["scale"], a["temp_n0"], a["dtype"], None)
+                                     a["scale"], a["temp_n0"], a["dtype"], a["ws"], a["ws_bytes"], None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -206,7 +215,10 @@ def _fwd_bank(lib, **kw):
     (dict(proj_heads=2), ops.RELBIAS_ERR_ARG),       # neither 1 nor Hq
     (dict(rs=None), ops.RELBIAS_ERR_ARG),
     (dict(proj=None), ops.RELBIAS_ERR_ARG),
-    (dict(dtype=ops.RELBIAS_BF16, d=128), ops.RELBIAS_ERR_UNSUPPORTED),   # bank runs on the fp32 path
+    (dict(dtype=ops.RELBIAS_BF16, d=128), ops.RELBIAS_ERR_ARG),           # bf16 bank needs its workspace
+    (dict(dtype=ops.RELBIAS_BF16, d=128, ws=FAKE + 16, ws_bytes=1 << 20), ops.RELBIAS_ERR_ARG),   # misaligned
+    (dict(dtype=ops.RELBIAS_BF16, d=128, ws=FAKE, ws_bytes=64), ops.RELBIAS_ERR_ARG),             # too small
+    (dict(dtype=ops.RELBIAS_BF16, d=96, ws=FAKE, ws_bytes=1 << 20), ops.RELBIAS_ERR_UNSUPPORTED),
     (dict(d=48), ops.RELBIAS_ERR_UNSUPPORTED),
 ])
 def test_fwd_bank_rejects_on_host(lib, kw, code):

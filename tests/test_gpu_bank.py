@@ -3,8 +3,9 @@
 The essay's recipe keeps a bank of C functions of distance shared by the heads of a
 layer, and gives each token and head C coefficients; the bias is their product
 ("Thinking Machines dropped RoPE", steps 1-2).  relbias_attn_fwd_bank runs it on the
-fp32 prefill path, relbias_attn_decode_bank on the bf16 split-KV decode (through
-per-(sequence, head) curves).  The oracle takes the same rs [.., C] and proj
+fp32 prefill path and on the bf16 tensor-core prefill (through per-row curves),
+relbias_attn_decode_bank on the bf16 split-KV decode (through per-(sequence, head)
+curves).  The oracle takes the same rs [.., C] and proj
 [1 or Hq, C, R] tensors.
 """
 import math
@@ -70,13 +71,85 @@ def test_fp32_bank_of_one_function_per_head_is_the_rank1_form_bitwise():
     assert torch.equal(o1, o2)
 
 
-def test_bf16_prefill_bank_is_unsupported():
-    x = {n: synth.normal((1, 128, 4, 128), 1, n, dtype=torch.bfloat16, device="cuda") for n in ("q", "k", "v")}
-    rs = synth.normal((1, 128, 4, 16), 1, "rs", device="cuda")
-    proj = synth.normal((1, 16, 64), 1, "proj", device="cuda")
-    with pytest.raises(ops.RelbiasError) as e:
-        ops.attn_fwd_bank(x["q"], x["k"], x["v"], rs, proj, 0, 64)
-    assert e.value.code == ops.RELBIAS_ERR_UNSUPPORTED
+BF16_CASES = [
+    # B, T,   Hq, Hkv, d,   window, R,   C,  proj_heads, temp_n0
+    (1, 200, 4, 2, 128, 0, 64, 16, 1, 0),       # the essay's 16-function bank, shared; ragged tail
+    (2, 300, 8, 2, 128, 128, 128, 16, 8, 0),    # a bank per head, windowed (local-layer form)
+    (1, 513, 6, 3, 64, 0, 300, 5, 1, 100),      # odd group, d = 64, temperature, R not a tile multiple
+    (1, 1, 4, 4, 128, 0, 16, 3, 1, 0),          # a single token
+    (1, 260, 4, 2, 128, 0, 1000, 16, 1, 0),     # R beyond the sequence
+]
+
+
+def _bank_inputs(B, T, Hq, Hkv, d, R, C, proj_heads, seed, dtype=torch.bfloat16):
+    dev = "cuda"
+    return (synth.normal((B, T, Hq, d), seed, "q", dtype=dtype, device=dev),
+            synth.normal((B, T, Hkv, d), seed, "k", dtype=dtype, device=dev),
+            synth.normal((B, T, Hkv, d), seed, "v", dtype=dtype, device=dev),
+            synth.normal((B, T, Hq, C), seed, "rs", std=1.0 / math.sqrt(C), device=dev),
+            synth.normal((proj_heads, C, R), seed, "proj", std=0.5, device=dev))
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,d,window,R,C,proj_heads,temp_n0", BF16_CASES)
+def test_bf16_prefill_bank_parity(B, T, Hq, Hkv, d, window, R, C, proj_heads, temp_n0):
+    """The tensor-core prefill with the bank's per-row curves, against the oracle's bank form."""
+    q, k, v, rs, proj = _bank_inputs(B, T, Hq, Hkv, d, R, C, proj_heads, seed=T + C + d)
+    scale = 1.0 / math.sqrt(d)
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd_bank(q, k, v, rs, proj, window, R, scale, lse=lse, temp_n0=temp_n0)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = O.attn_prefill(q.cpu(), k.cpu(), v.cpu(), rs.cpu(), proj.cpu(), window, R, scale,
+                                    temp_n0=temp_n0)
+    assert_bf16_close(o, o_ref, lse, lse_ref, "bf16 bank %s" % ((B, T, Hq, Hkv, d, window, R, C, proj_heads),))
+
+
+def test_bf16_bank_of_one_function_per_head_matches_rank1():
+    """C = 1 with a bank per head is the rank-1 form; the two bf16 paths agree to rounding
+    (the bank path forms r * w in its curve kernel, the rank-1 path in the softmax)."""
+    B, T, Hq, Hkv, d, R = 2, 300, 8, 2, 128, 200
+    dev = "cuda"
+    q = synth.normal((B, T, Hq, d), 12, "q", dtype=torch.bfloat16, device=dev)
+    k = synth.normal((B, T, Hkv, d), 12, "k", dtype=torch.bfloat16, device=dev)
+    v = synth.normal((B, T, Hkv, d), 12, "v", dtype=torch.bfloat16, device=dev)
+    r = synth.normal((B, T, Hq), 12, "r", device=dev)
+    w = synth.normal((Hq, R), 12, "w", std=0.5, device=dev)
+    l1 = torch.empty(B, Hq, T, dtype=torch.float32, device=dev)
+    l2 = torch.empty_like(l1)
+    o1 = ops.attn_fwd(q, k, v, r, w, 128, R, 0.09, lse=l1)
+    o2 = ops.attn_fwd_bank(q, k, v, r[..., None].contiguous(), w[:, None, :].contiguous(), 128, R, 0.09, lse=l2)
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_bf16_bank_workspace_is_not_read_before_written():
+    """The curve workspace's prior contents do not matter (NaN-filled here)."""
+    B, T, Hq, Hkv, d, R, C = 1, 257, 4, 2, 128, 100, 16
+    q, k, v, rs, proj = _bank_inputs(B, T, Hq, Hkv, d, R, C, 1, seed=77)
+    need = ops.fwd_bank_workspace_size(B, T, Hq, R, ops.RELBIAS_BF16)
+    ws = torch.full((need // 4,), float("nan"), dtype=torch.float32, device="cuda").view(torch.uint8)
+    o = ops.attn_fwd_bank(q, k, v, rs, proj, 0, R, 0.1, workspace=ws)
+    torch.cuda.synchronize()
+    o_ref, _ = O.attn_prefill(q.cpu(), k.cpu(), v.cpu(), rs.cpu(), proj.cpu(), 0, R, 0.1)
+    assert_bf16_close(o, o_ref, what="bf16 bank, NaN-filled workspace")
+
+
+def test_bf16_prefill_bank_workload_sampled():
+    """The local-layer shape with the essay's 16-function shared bank, in the launch
+    configuration the benchmark times, on sampled rows."""
+    from parity import sample_rows
+    wl = WORKLOADS["local_prefill_bank_bf16"]
+    x = make_inputs(wl, device="cuda")
+    B, T, Hq, d = x["q"].shape
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], wl.window, wl.R, wl.scale, lse=lse)
+    torch.cuda.synchronize()
+    rows = sample_rows(B, T, Hq, per_head=3, seed=5, extra=(8190,))
+    o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["rs"].cpu(), x["proj"].cpu(),
+                                    wl.window, wl.R, wl.scale, rows=rows)
+    got = o.float().cpu()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    got_lse = lse.cpu()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert_bf16_close(got, o_ref, got_lse, lse_ref, wl.name)
 
 
 DECODE_CASES = [
