@@ -1,0 +1,824 @@
+// backward_sm100.cu -- gradients of the biased attention forward pass on the tcgen05
+// tensor cores (bf16 inputs, fp32 accumulation in tensor memory).
+//
+// For one row (b, h, i) with logits l_j = tau_i * (scale * q_i.k_j + r_i * w[h, i-j])
+// over the attended keys, p_j = exp(l_j - LSE_i) and D_i = dO_i.O_i, the derivative
+// of the loss with respect to l_j is dl_j = p_j (dO_i.v_j - D_i), and
+//   dq_i = tau_i scale sum_j dl_j k_j        dk_j = sum_(h,i) tau_i scale dl_j q_i
+//   dv_j = sum_(h,i) p_j dO_i                 dr_i = tau_i sum_j dl_j w[h, i-j]
+//   dw[h, d] = sum_i tau_i dl_(i, i-d) r_i
+// (the plain derivative of the forward definition: "Thinking Machines dropped RoPE",
+// recipe steps 3-5, for the bias; the pages train the model but print no backward).
+//
+// Two kernels, as in the forward one row of a 128 x 128 tile per thread:
+//   bwd_dq_sm100_kernel    per (sequence, query head, 128-row query tile): over the
+//       visible key tiles, S = Q K^T and dP = dO V^T into tensor memory, dl in
+//       registers (dr accumulated with the staged distance table, as the forward adds
+//       the bias), dS = tau scale dl written back over S as bf16, dQ += dS K.  Writes
+//       dq, dr and D_i (for the second kernel).
+//   bwd_dkv_sm100_kernel   per (sequence, key/value head, 128-key tile): over the
+//       group's query heads and the query tiles that see the keys, S^T = K Q^T and
+//       dP^T = V dO^T, P^T and dS^T in registers (one key row per thread), then
+//       dV += P^T dO and dK += dS^T Q with P^T and dS^T read from tensor memory; dw
+//       summed along the tile's diagonals in shared memory.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace relbias {
+
+namespace {
+
+// ------------------------------------------------------------------------- dQ kernel
+
+constexpr int kBqThreads = 192;   // warps 0-3 rows, 4 TMA producer, 5 MMA issuer
+
+template <int D>
+struct BqLayout {
+    static constexpr int kTile = kBM * D * 2;
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTile;
+    static constexpr int kK = kDO + kTile;             // 2 stages
+    static constexpr int kV = kK + 2 * kTile;          // 2 stages
+    static constexpr int kTab = kV + 2 * kTile;
+};
+
+struct BqBars {
+    uint64_t q_full, q_empty, do_full, do_empty;
+    uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+    uint64_t sdp_full;     // S(g) and dP(g) complete
+    uint64_t dp_free;      // the rows' warps hold dP(g) in registers
+    uint64_t ds_ready;     // dS(g) is in tensor memory
+    uint64_t dq_final;     // an item's last dQ MMA complete
+    uint64_t dq_free;      // the rows' warps have read an item's dQ
+    uint64_t tab_sync;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+int bq_smem_bytes(int d, int R, int ncopy) {
+    const int lay = d == 64 ? BqLayout<64>::kTab : BqLayout<128>::kTab;
+    return lay + tab_floats(R, ncopy) * 4 + static_cast<int>(sizeof(BqBars)) + 1024;
+}
+
+// The tile stream of a CTA: item by item, key tile by key tile.
+struct TileCursor {
+    int item_it, nitems, t, ntiles, j_first;
+    Item it;
+    __device__ __forceinline__ void load(const PrefillParams& p) {
+        it = item_at(p, item_it);
+        kv_range(p, it.qt * kBM, j_first, ntiles);
+        t = 0;
+    }
+    __device__ __forceinline__ bool next(const PrefillParams& p) {
+        if (++t < ntiles) return true;
+        if (++item_it >= nitems) return false;
+        load(p);
+        return true;
+    }
+    __device__ __forceinline__ bool first() const { return t == 0; }
+    __device__ __forceinline__ bool last() const { return t == ntiles - 1; }
+    __device__ __forceinline__ int j0() const { return j_first + t * kBN; }
+};
+
+template <int D, int NCOPY>
+__global__ void __launch_bounds__(kBqThreads, 1)
+    bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const PrefillParams p, const BwdTcParams bp) {
+    using L = BqLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tstride = tab_stride(p.R, NCOPY);
+    const int tslot = NCOPY * tstride;
+    float* wtab = reinterpret_cast<float*>(smem + L::kTab);
+    BqBars* bars = reinterpret_cast<BqBars*>(smem + L::kTab + tslot * 4);
+    volatile int* abort_flag = &bars->abort_flag;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->do_full, 1);
+        mbar_init(&bars->do_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        mbar_init(&bars->sdp_full, 1);
+        mbar_init(&bars->dp_free, kBM / 32);
+        mbar_init(&bars->ds_ready, kBM / 32);
+        mbar_init(&bars->dq_final, 1);
+        mbar_init(&bars->dq_free, kBM / 32);
+        mbar_init(&bars->tab_sync, kBM / 32);
+        mbar_init(&bars->mma_done, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_base;
+    const int nitems = items_of_cta(p);
+    // Tensor memory: S(g) in [128 * (g & 1), +128), dP [256, 384), dQ [384, 384 + D).
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        const bool leader = elect_one();
+        bool ok = true;
+        int nq = 0, nkv = 0;   // items and key tiles whose copies were issued
+        int g = 0;
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const Item it = item_at(p, item_it);
+            const int i0 = it.qt * kBM;
+            int j_first, ntiles;
+            kv_range(p, i0, j_first, ntiles);
+            const int h = it.g * p.G + it.hp;
+            if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->q_empty, (item_it - 1) & 1, abort_flag)))) break;
+            if (leader) {
+                mbar_arrive_expect_tx(&bars->q_full, L::kTile);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(smem + L::kQ + bx * kBM * 128, &tm_q, &bars->q_full, bx * 64, h, i0, it.b);
+            }
+            if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->do_empty, (item_it - 1) & 1, abort_flag)))) break;
+            if (leader) {
+                mbar_arrive_expect_tx(&bars->do_full, L::kTile);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(smem + L::kDO + bx * kBM * 128, &tm_do, &bars->do_full, bx * 64, h, i0, it.b);
+            }
+            ++nq;
+            for (int t = 0; t < ntiles; ++t, ++g) {
+                const int st = g & 1;
+                const uint32_t ph = (g >> 1) & 1;
+                const int j0 = j_first + t * kBN;
+                if (!(ok = warp_all(mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag)))) break;
+                if (!(ok = warp_all(mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag)))) break;
+                if (leader) {
+                    mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
+                    mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
+                    for (int bx = 0; bx < D / 64; ++bx) {
+                        tma_load_4d(smem + L::kK + st * L::kTile + bx * kBM * 128, &tm_k, &bars->k_full[st],
+                                    bx * 64, it.g, j0, it.b);
+                        tma_load_4d(smem + L::kV + st * L::kTile + bx * kBM * 128, &tm_v, &bars->v_full[st],
+                                    bx * 64, it.g, j0, it.b);
+                    }
+                }
+                ++nkv;
+            }
+        }
+        // Drain, also after an abort: no copy into this CTA's shared memory may be in flight
+        // when it exits.  Each barrier has at most its last phase outstanding.
+        if (nq > 0) {
+            mbar_drain_wait(&bars->q_full, (nq - 1) & 1);
+            mbar_drain_wait(&bars->do_full, (nq - 1) & 1);
+        }
+        for (int n = max(0, nkv - 2); n < nkv; ++n) {
+            mbar_drain_wait(&bars->k_full[n & 1], (n >> 1) & 1);
+            mbar_drain_wait(&bars->v_full[n & 1], (n >> 1) & 1);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        // Per tile g the issue order is QK(g+1), dP(g+1), dQ(g): the next tile's S and dP
+        // are computed while the rows' warps work on tile g (S is double-buffered; dP is
+        // rewritten once the warps hold dP(g) in registers).
+        const bool leader = elect_one();
+        const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
+        const uint32_t idesc_dq = idesc_bf16_f32(kBM, D, false, true);
+        const uint32_t dp_tm = tmem_base + 256, dq_tm = tmem_base + 384;
+        const uint32_t q_addr = smem_u32(smem + L::kQ), do_addr = smem_u32(smem + L::kDO);
+        bool ok = nitems > 0;
+        TileCursor cur{0, nitems, 0, 0, 0, {}};
+        if (ok) cur.load(p);
+        // Issue QK and dP of tile g (its stage st); first tiles of an item wait for Q / dO.
+        auto issue_s_dp = [&](const TileCursor& c, int g, bool wait_dp_free) -> bool {
+            const int st = g & 1;
+            const uint32_t ph = (g >> 1) & 1;
+            if (!warp_all(mbar_wait(&bars->k_full[st], ph, abort_flag))) return false;
+            if (c.first() && !warp_all(mbar_wait(&bars->q_full, c.item_it & 1, abort_flag))) return false;
+            tc_fence_after();
+            issue_qk<D>(leader, tmem_base + 128 * (g & 1), q_addr, smem_u32(smem + L::kK + st * L::kTile), idesc_qk);
+            if (leader && c.last()) umma_commit(&bars->q_empty);
+            if (wait_dp_free && !warp_all(mbar_wait(&bars->dp_free, (g - 1) & 1, abort_flag))) return false;
+            if (!warp_all(mbar_wait(&bars->v_full[st], ph, abort_flag))) return false;
+            if (c.first() && !warp_all(mbar_wait(&bars->do_full, c.item_it & 1, abort_flag))) return false;
+            tc_fence_after();
+            issue_qk<D>(leader, dp_tm, do_addr, smem_u32(smem + L::kV + st * L::kTile), idesc_qk);
+            if (leader) umma_commit(&bars->v_empty[st]);
+            if (leader && c.last()) umma_commit(&bars->do_empty);
+            if (leader) umma_commit(&bars->sdp_full);
+            return true;
+        };
+        if (ok) ok = issue_s_dp(cur, 0, false);
+        for (int g = 0; ok; ++g) {
+            TileCursor nxt = cur;
+            const bool have_next = nxt.next(p);
+            if (have_next && !(ok = issue_s_dp(nxt, g + 1, true))) break;
+            if (!(ok = warp_all(mbar_wait(&bars->ds_ready, g & 1, abort_flag)))) break;
+            if (cur.first() && cur.item_it > 0 &&
+                !(ok = warp_all(mbar_wait(&bars->dq_free, (cur.item_it - 1) & 1, abort_flag))))
+                break;
+            tc_fence_after();
+            // dQ += dS K: dS (bf16 pairs over the first 64 columns of S(g)) times the key tile,
+            // keys on the K dimension (MN-major operand, as V in the forward's PV).
+            issue_pv<D>(leader, dq_tm, tmem_base + 128 * (g & 1), smem_u32(smem + L::kK + (g & 1) * L::kTile),
+                        idesc_dq, !cur.first());
+            if (leader) umma_commit(&bars->k_empty[g & 1]);
+            if (leader && cur.last()) umma_commit(&bars->dq_final);
+            if (!have_next) break;
+            cur = nxt;
+        }
+        if (leader) umma_commit(&bars->mma_done);
+        mbar_drain_wait(&bars->mma_done, 0);
+    } else {
+        // ---------------------------------------------------------------- rows
+        const int t = threadIdx.x;                       // row t of the query tile (TMEM lane)
+        const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
+        const uint32_t dp_tm = tmem_base + lane_off + 256, dq_tm = tmem_base + lane_off + 384;
+        const int cmax = tab_cmax(p.R);
+        int staged_head = -1;
+        uint32_t tab_phase = 0;
+        int g = 0;
+        bool ok = true;
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const Item it = item_at(p, item_it);
+            const int i0 = it.qt * kBM;
+            int j_first, ntiles;
+            kv_range(p, i0, j_first, ntiles);
+            const int h = it.g * p.G + it.hp;
+            if (h != staged_head) {
+                staged_head = h;
+                if (!(ok = tab_meet(&bars->tab_sync, tab_phase, abort_flag))) break;
+                const float* wrow = p.w + static_cast<size_t>(h) * p.R;
+                for (int x = t; x < tslot; x += kBM) {
+                    const int cp = x / tstride;
+                    const int dd = cmax - (x - cp * tstride + cp);
+                    wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(wrow + dd) : 0.0f;
+                }
+                if (!(ok = tab_meet(&bars->tab_sync, tab_phase, abort_flag))) break;
+            }
+            const int i = i0 + t;
+            const bool row_ok = i < p.T;
+            const size_t row = (static_cast<size_t>(it.b) * p.T + (row_ok ? i : 0)) * p.Hq + h;   // [B, T, Hq]
+            const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + (row_ok ? i : 0);  // [B, Hq, T]
+            // D_i = dO_i . O_i, the row's log-sum-exp in log2 units, the logit scale with
+            // the context-length temperature, and the bias coefficient (log2 units).
+            float Di = 0.0f;
+            if (row_ok) {
+                const uint4* orow = reinterpret_cast<const uint4*>(bp.o + row * D);
+                const uint4* grow = reinterpret_cast<const uint4*>(bp.dout + row * D);
+#pragma unroll 4
+                for (int u = 0; u < D / 8; ++u) {
+                    const uint4 a = __ldg(orow + u), b = __ldg(grow + u);
+                    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+                        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+                        Di = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, Di));
+                    }
+                }
+                bp.dvec[hrow] = Di;
+            }
+            const float lse2 = row_ok ? __ldg(bp.lse + hrow) * 1.4426950408889634f : 0.0f;
+            float tau = 1.0f;
+            if (p.temp_n0 > 1) {
+                const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
+                if (n > p.temp_n0) tau = __logf(static_cast<float>(n)) * p.inv_log_n0;
+            }
+            const float c1 = p.scale_log2 * tau;
+            const float rb = row_ok ? __ldg(p.r + row) * p.inv_scale * c1 : 0.0f;   // bias, log2 units
+            const float ds_scale = tau * bp.scale;   // dS = tau * scale * dl, the dQ MMA's operand
+            float dr_acc = 0.0f;                     // sum_j dl_j w[h, i-j]
+
+            for (int tt = 0; tt < ntiles; ++tt, ++g) {
+                const int j0 = j_first + tt * kBN;
+                const int delta0 = i0 - j0;
+                const uint32_t s_tm = tmem_base + lane_off + 128 * (g & 1);
+                if (!(ok = warp_all(mbar_wait(&bars->sdp_full, g & 1, abort_flag)))) break;
+                tc_fence_after();
+                uint32_t dp[kBN];
+#pragma unroll
+                for (int c = 0; c < kBN; c += 32) tmem_ld32(dp_tm + c, dp + c);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dp_free);
+                const bool biased = delta0 - (kBN - 1) < p.R;
+                const int base = cmax - delta0 - t;
+                const int cp = base & (NCOPY - 1);
+                const float* run = wtab + cp * tstride + (base - cp);
+                const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window);
+                const int hi = delta0 + t;
+                const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
+#pragma unroll
+                for (int ch = 0; ch < kBN / 32; ++ch) {
+                    uint32_t sv[32];
+                    tmem_ld32(s_tm + 32 * ch, sv);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        float w4[4] = {0.f, 0.f, 0.f, 0.f};
+                        if (biased) {
+                            if constexpr (NCOPY == 4) {
+                                const float4 v = *reinterpret_cast<const float4*>(run + 32 * ch + e);
+                                w4[0] = v.x, w4[1] = v.y, w4[2] = v.z, w4[3] = v.w;
+                            } else if constexpr (NCOPY == 2) {
+                                const float2 a = *reinterpret_cast<const float2*>(run + 32 * ch + e);
+                                const float2 b = *reinterpret_cast<const float2*>(run + 32 * ch + e + 2);
+                                w4[0] = a.x, w4[1] = a.y, w4[2] = b.x, w4[3] = b.y;
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) w4[k] = run[32 * ch + e + k];
+                            }
+                        }
+                        float dl[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int c = 32 * ch + e + k;
+                            const float x = fmaf(__uint_as_float(sv[e + k]), c1, fmaf(rb, w4[k], -lse2));
+                            const bool vis = !edge || (c <= hi && c >= lo);
+                            const float pr = vis ? ex2_approx(x) : 0.0f;
+                            dl[k] = pr * (__uint_as_float(dp[c]) - Di);
+                            dr_acc = fmaf(dl[k], w4[k], dr_acc);
+                        }
+                        pk[e / 2] = pack_bf16x2(dl[0] * ds_scale, dl[1] * ds_scale);
+                        pk[e / 2 + 1] = pack_bf16x2(dl[2] * ds_scale, dl[3] * ds_scale);
+                    }
+                    tmem_st16(s_tm + 16 * ch, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->ds_ready);
+            }
+            if (!ok) break;
+
+            // Epilogue: dr and the row of dq.
+            if (row_ok) bp.dr[row] = dr_acc * tau;
+            if (!(ok = warp_all(mbar_wait(&bars->dq_final, item_it & 1, abort_flag)))) break;
+            tc_fence_after();
+            float* dqrow = bp.dq + row * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+                uint32_t v[32];
+                tmem_ld32(dq_tm + c, v);
+                tmem_ld_wait();
+                if (row_ok) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(dqrow + c + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                        __uint_as_float(v[e + 3]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dq_free);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+
+// ------------------------------------------------------------------------- dK/dV kernel
+
+constexpr int kBkThreads = 192;   // warps 0-3 key rows, 4 TMA producer, 5 MMA issuer
+
+template <int D>
+struct BkLayout {
+    static constexpr int kTile = kBM * D * 2;
+    static constexpr int kK = 0;
+    static constexpr int kV = kK + kTile;
+    static constexpr int kQ = kV + kTile;              // 2 stages
+    static constexpr int kDO = kQ + 2 * kTile;         // 2 stages
+    static constexpr int kCol = kDO + 2 * kTile;       // per-column constants, 2 buffers of [128] float8
+    static constexpr int kDw = kCol + 2 * kBM * 32;    // table gradient accumulator [R]
+};
+
+struct BkBars {
+    uint64_t kv_full, kv_empty;
+    uint64_t q_full[2], q_empty[2], do_full[2], do_empty[2];
+    uint64_t sdp_full;     // S^T(s) and dP^T(s) complete
+    uint64_t pd_ready;     // P^T(s) and dS^T(s) are in tensor memory
+    uint64_t acc_final;    // an item's last dK / dV MMA complete
+    uint64_t acc_free;     // the rows' warps have read an item's dK and dV
+    uint64_t col_sync;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// Non-reversed distance table: entry y <-> distance y - 265 (zeros outside [0, R)),
+// NCOPY copies shifted by one entry; a key row's run over the 128 query columns of a
+// tile is ascending.
+constexpr int kBkDmin = -265;
+
+int bk_smem_bytes(int d, int R, int ncopy) {
+    const int lay = d == 64 ? BkLayout<64>::kDw : BkLayout<128>::kDw;
+    return lay + ((R + 3) / 4) * 16 + tab_floats(R, ncopy) * 4 + static_cast<int>(sizeof(BkBars)) + 1024;
+}
+
+// Query tiles that see key tile kt: [qt_lo, qt_hi].
+__device__ __forceinline__ void q_range(const PrefillParams& p, int kt, int& qt_lo, int& qt_hi) {
+    const int k0 = kt * kBN;
+    qt_lo = k0 / kBM;
+    const int last_row = p.window > 0 ? min(p.T - 1, k0 + kBN - 1 + p.window - 1) : p.T - 1;
+    qt_hi = last_row / kBM;
+}
+
+// Items: (b, key/value head g, key tile), heaviest (earliest) key tiles first for causal
+// layers, runs of consecutive key tiles for windowed ones.
+struct BkItem {
+    int kt, b, g;
+};
+__device__ __forceinline__ int bk_items_of_cta(const PrefillParams& p) {
+    if (p.contiguous) {
+        const int per = (p.total_items + gridDim.x - 1) / gridDim.x;
+        return max(0, min(per, p.total_items - static_cast<int>(blockIdx.x) * per));
+    }
+    return (p.total_items - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
+}
+__device__ __forceinline__ BkItem bk_item_at(const PrefillParams& p, int k) {
+    BkItem it;
+    if (p.contiguous) {
+        const int per = (p.total_items + gridDim.x - 1) / gridDim.x;
+        const int u = static_cast<int>(blockIdx.x) * per + k;
+        it.kt = u % p.n_qt;
+        const int rem = u / p.n_qt;
+        it.g = rem % p.Hkv;
+        it.b = rem / p.Hkv;
+        return it;
+    }
+    const int u = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+    const int per_kt = p.B * p.Hkv;
+    it.kt = u / per_kt;
+    const int rem = u - it.kt * per_kt;
+    it.b = rem / p.Hkv;
+    it.g = rem - it.b * p.Hkv;
+    return it;
+}
+
+template <int D, int NCOPY>
+__global__ void __launch_bounds__(kBkThreads, 1)
+    bwd_dkv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const PrefillParams p, const BwdTcParams bp) {
+    using L = BkLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tstride = tab_stride(p.R, NCOPY);
+    const int tslot = NCOPY * tstride;
+    float* dw_s = reinterpret_cast<float*>(smem + L::kDw);
+    const int dw_len = ((p.R + 3) / 4) * 4;
+    float* wtab = dw_s + dw_len;
+    BkBars* bars = reinterpret_cast<BkBars*>(reinterpret_cast<uint8_t*>(wtab) + tslot * 4);
+    volatile int* abort_flag = &bars->abort_flag;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        mbar_init(&bars->kv_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+            mbar_init(&bars->do_full[s], 1);
+            mbar_init(&bars->do_empty[s], 1);
+        }
+        mbar_init(&bars->sdp_full, 1);
+        mbar_init(&bars->pd_ready, kBM / 32);
+        mbar_init(&bars->acc_final, 1);
+        mbar_init(&bars->acc_free, kBM / 32);
+        mbar_init(&bars->col_sync, kBM / 32);
+        mbar_init(&bars->mma_done, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_base;
+    const int nitems = bk_items_of_cta(p);
+    // Tensor memory: S^T [0, 128) (P^T over it), dP^T [128, 256) (dS^T over it),
+    // dV [256, 256 + D), dK [384, 384 + D).  Steps s run over (head of the group, query
+    // tile) within an item, and across items.
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        const bool leader = elect_one();
+        bool ok = true;
+        int nkv = 0, ns = 0;
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const BkItem it = bk_item_at(p, item_it);
+            const int k0 = it.kt * kBN;
+            int qt_lo, qt_hi;
+            q_range(p, it.kt, qt_lo, qt_hi);
+            if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->kv_empty, (item_it - 1) & 1, abort_flag)))) break;
+            if (leader) {
+                mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
+                for (int bx = 0; bx < D / 64; ++bx) {
+                    tma_load_4d(smem + L::kK + bx * kBM * 128, &tm_k, &bars->kv_full, bx * 64, it.g, k0, it.b);
+                    tma_load_4d(smem + L::kV + bx * kBM * 128, &tm_v, &bars->kv_full, bx * 64, it.g, k0, it.b);
+                }
+            }
+            ++nkv;
+            for (int hl = 0; ok && hl < p.G; ++hl) {
+                const int h = it.g * p.G + hl;
+                for (int qt = qt_lo; qt <= qt_hi; ++qt, ++ns) {
+                    const int st = ns & 1;
+                    const uint32_t ph = (ns >> 1) & 1;
+                    if (!(ok = warp_all(mbar_wait(&bars->q_empty[st], ph ^ 1, abort_flag)))) break;
+                    if (!(ok = warp_all(mbar_wait(&bars->do_empty[st], ph ^ 1, abort_flag)))) break;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&bars->q_full[st], L::kTile);
+                        mbar_arrive_expect_tx(&bars->do_full[st], L::kTile);
+                        for (int bx = 0; bx < D / 64; ++bx) {
+                            tma_load_4d(smem + L::kQ + st * L::kTile + bx * kBM * 128, &tm_q, &bars->q_full[st],
+                                        bx * 64, h, qt * kBM, it.b);
+                            tma_load_4d(smem + L::kDO + st * L::kTile + bx * kBM * 128, &tm_do, &bars->do_full[st],
+                                        bx * 64, h, qt * kBM, it.b);
+                        }
+                    }
+                }
+            }
+        }
+        if (nkv > 0) mbar_drain_wait(&bars->kv_full, (nkv - 1) & 1);
+        for (int n = max(0, ns - 2); n < ns; ++n) {
+            mbar_drain_wait(&bars->q_full[n & 1], (n >> 1) & 1);
+            mbar_drain_wait(&bars->do_full[n & 1], (n >> 1) & 1);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        const bool leader = elect_one();
+        const uint32_t idesc_s = idesc_bf16_f32(kBM, kBM, false, false);
+        const uint32_t idesc_acc = idesc_bf16_f32(kBN, D, false, true);
+        const uint32_t st_tm = tmem_base, dpt_tm = tmem_base + 128, dv_tm = tmem_base + 256,
+                       dk_tm = tmem_base + 384;
+        const uint32_t k_addr = smem_u32(smem + L::kK), v_addr = smem_u32(smem + L::kV);
+        bool ok = true;
+        int ns = 0;
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const BkItem it = bk_item_at(p, item_it);
+            int qt_lo, qt_hi;
+            q_range(p, it.kt, qt_lo, qt_hi);
+            const int nsteps = p.G * (qt_hi - qt_lo + 1);
+            if (!(ok = warp_all(mbar_wait(&bars->kv_full, item_it & 1, abort_flag)))) break;
+            if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->acc_free, (item_it - 1) & 1, abort_flag)))) break;
+            for (int s = 0; s < nsteps; ++s, ++ns) {
+                const int st = ns & 1;
+                const uint32_t ph = (ns >> 1) & 1;
+                const uint32_t q_addr = smem_u32(smem + L::kQ + st * L::kTile);
+                const uint32_t do_addr = smem_u32(smem + L::kDO + st * L::kTile);
+                if (!(ok = warp_all(mbar_wait(&bars->q_full[st], ph, abort_flag)))) break;
+                if (!(ok = warp_all(mbar_wait(&bars->do_full[st], ph, abort_flag)))) break;
+                tc_fence_after();
+                // S^T = K Q^T and dP^T = V dO^T (keys on M, query rows on N).
+                issue_qk<D>(leader, st_tm, k_addr, q_addr, idesc_s);
+                issue_qk<D>(leader, dpt_tm, v_addr, do_addr, idesc_s);
+                if (leader) umma_commit(&bars->sdp_full);
+                if (!(ok = warp_all(mbar_wait(&bars->pd_ready, ns & 1, abort_flag)))) break;
+                tc_fence_after();
+                // dV += P^T dO and dK += dS^T Q: query rows on the K dimension.
+                issue_pv<D>(leader, dv_tm, st_tm, do_addr, idesc_acc, s > 0);
+                issue_pv<D>(leader, dk_tm, dpt_tm, q_addr, idesc_acc, s > 0);
+                if (leader) {
+                    umma_commit(&bars->q_empty[st]);
+                    umma_commit(&bars->do_empty[st]);
+                }
+            }
+            if (!ok) break;
+            if (leader) {
+                umma_commit(&bars->kv_empty);
+                umma_commit(&bars->acc_final);
+            }
+        }
+        if (leader) umma_commit(&bars->mma_done);
+        mbar_drain_wait(&bars->mma_done, 0);
+    } else {
+        // ---------------------------------------------------------------- key rows
+        const int t = threadIdx.x;   // key k0 + t of the tile (TMEM lane)
+        const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
+        const uint32_t st_tm = tmem_base + lane_off, dpt_tm = tmem_base + lane_off + 128,
+                       dv_tm = tmem_base + lane_off + 256, dk_tm = tmem_base + lane_off + 384;
+        float4* col = reinterpret_cast<float4*>(smem + L::kCol);   // [2][128] x {c1, rb, lse2, D, dsc, twr, -, -}
+        uint32_t col_phase = 0;
+        int ns = 0;
+        bool ok = true;
+        for (int item_it = 0; ok && item_it < nitems; ++item_it) {
+            const BkItem it = bk_item_at(p, item_it);
+            const int k0 = it.kt * kBN;
+            const int j = k0 + t;
+            const bool key_ok = j < p.T;
+            int qt_lo, qt_hi;
+            q_range(p, it.kt, qt_lo, qt_hi);
+            for (int hl = 0; ok && hl < p.G; ++hl) {
+                const int h = it.g * p.G + hl;
+                // This head's table (ascending) and a zeroed dw accumulator.
+                if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
+                if (p.R > 0) {
+                    const float* wrow = p.w + static_cast<size_t>(h) * p.R;
+                    for (int x = t; x < tslot; x += kBM) {
+                        const int cp = x / tstride;
+                        const int dd = x - cp * tstride + cp + kBkDmin;
+                        wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(wrow + dd) : 0.0f;
+                    }
+                    for (int x = t; x < dw_len; x += kBM) dw_s[x] = 0.0f;
+                }
+                for (int qt = qt_lo; qt <= qt_hi; ++qt, ++ns) {
+                    const int i0 = qt * kBM;
+                    float4* cb = col + (ns & 1) * 2 * kBM;
+                    {
+                        // Column constants of query row i0 + t (this thread fills column t).
+                        const int i = i0 + t;
+                        const bool row_ok = i < p.T;
+                        const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + (row_ok ? i : 0);
+                        float tau = 1.0f;
+                        if (p.temp_n0 > 1) {
+                            const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
+                            if (n > p.temp_n0) tau = __logf(static_cast<float>(n)) * p.inv_log_n0;
+                        }
+                        const float c1 = p.scale_log2 * tau;
+                        const float ri = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) : 0.0f;
+                        const float lse2 = row_ok ? __ldg(bp.lse + hrow) * 1.4426950408889634f : 0.0f;
+                        const float Di = row_ok ? bp.dvec[hrow] : 0.0f;
+                        cb[2 * t] = make_float4(c1, ri * p.inv_scale * c1, lse2, Di);
+                        cb[2 * t + 1] = make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
+                    }
+                    if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
+                    if (!(ok = warp_all(mbar_wait(&bars->sdp_full, ns & 1, abort_flag)))) break;
+                    tc_fence_after();
+                    const int delta0 = i0 - k0;                // distance of (key t, column c) is delta0 + c - t
+                    const bool biased = delta0 - (kBN - 1) < p.R;
+                    const int y0 = delta0 - t - kBkDmin;       // table entry of column 0
+                    const int cp = y0 & (NCOPY - 1);
+                    const float* run = wtab + cp * tstride + (y0 - cp);
+                    const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBN - 1 >= p.window);
+#pragma unroll 1
+                    for (int ch = 0; ch < kBM / 32; ++ch) {
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(st_tm + 32 * ch, sv);
+                        tmem_ld32(dpt_tm + 32 * ch, dv);
+                        tmem_ld_wait();
+                        uint32_t pp[16], pd[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float pr[2], dsv[2];
+#pragma unroll
+                            for (int k = 0; k < 2; ++k) {
+                                const int c = 32 * ch + e + k;
+                                const float4 a = cb[2 * c];
+                                const float4 b2 = cb[2 * c + 1];
+                                const int dist = delta0 + c - t;
+                                const float wv = biased ? run[c] : 0.0f;
+                                const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
+                                const bool vis = key_ok && dist >= 0 && i0 + c < p.T && (!edge || p.window <= 0 || dist < p.window);
+                                const float pv = vis ? ex2_approx(x) : 0.0f;
+                                const float dl = pv * (__uint_as_float(dv[e + k]) - a.w);
+                                pr[k] = pv;
+                                dsv[k] = dl * b2.x;
+                                if (biased && dist >= 0 && dist < p.R && dl != 0.0f) atomicAdd(dw_s + dist, dl * b2.y);
+                            }
+                            pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
+                            pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                        }
+                        tmem_st16(st_tm + 16 * ch, pp);
+                        tmem_st16(dpt_tm + 16 * ch, pd);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->pd_ready);
+                }
+                if (!ok) break;
+                // This head's table gradient from this key tile, into the output.
+                if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
+                for (int x = t; x < p.R; x += kBM)
+                    if (dw_s[x] != 0.0f) atomicAdd(bp.dw + static_cast<size_t>(h) * p.R + x, dw_s[x]);
+            }
+            if (!ok) break;
+            // Epilogue: the key row's dk and dv (fp32).
+            if (!(ok = warp_all(mbar_wait(&bars->acc_final, item_it & 1, abort_flag)))) break;
+            tc_fence_after();
+            const size_t krow = (static_cast<size_t>(it.b) * p.T + (key_ok ? j : 0)) * p.Hkv + it.g;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(dk_tm + c, a);
+                tmem_ld32(dv_tm + c, b);
+                tmem_ld_wait();
+                if (key_ok) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        *reinterpret_cast<float4*>(bp.dk + krow * D + c + e) = make_float4(
+                            __uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
+                            __uint_as_float(a[e + 3]));
+                        *reinterpret_cast<float4*>(bp.dv + krow * D + c + e) = make_float4(
+                            __uint_as_float(b[e]), __uint_as_float(b[e + 1]), __uint_as_float(b[e + 2]),
+                            __uint_as_float(b[e + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_free);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+template <int D>
+int bq_copies(int R) {
+    for (int nc = 4; nc >= 1; nc >>= 1)
+        if (bq_smem_bytes(D, R, nc) <= kMaxDynSmem) return nc;
+    return 0;
+}
+
+template <int D, int NCOPY>
+cudaError_t launch_bq(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const PrefillParams& p, const BwdTcParams& bp, int grid, cudaStream_t stream) {
+    auto kern = bwd_dq_sm100_kernel<D, NCOPY>;
+    // More than half of an SM's shared memory: one CTA (and one 512-column TMEM allocation) per SM.
+    const int smem = std::max(bq_smem_bytes(D, p.R, NCOPY), 120 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kBqThreads, smem, stream>>>(tq, tdo, tk, tv, p, bp);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bk(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const PrefillParams& p, const BwdTcParams& bp, int grid, cudaStream_t stream) {
+    auto kern = bwd_dkv_sm100_kernel<D, 1>;
+    const int smem = std::max(bk_smem_bytes(D, p.R, 1), 120 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kBkThreads, smem, stream>>>(tq, tdo, tk, tv, p, bp);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
+                          const BwdTcParams& bp, int grid, cudaStream_t stream) {
+    const int nc = bq_copies<D>(p_dq.R);
+    cudaError_t e = nc == 4   ? launch_bq<D, 4>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)
+                    : nc == 2 ? launch_bq<D, 2>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)
+                              : launch_bq<D, 1>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream);
+    if (e != cudaSuccess) return e;
+    return launch_bk<D>(tq, tdo, tk, tv, p_dkv, bp, std::min(grid, p_dkv.total_items), stream);
+}
+
+}  // namespace
+
+bool backward_tc_supported(int d, int R) {
+    if (d == 128) return bq_copies<128>(R) > 0 && bk_smem_bytes(128, R, 1) <= kMaxDynSmem;
+    if (d == 64) return bq_copies<64>(R) > 0 && bk_smem_bytes(64, R, 1) <= kMaxDynSmem;
+    return false;
+}
+
+cudaError_t launch_backward_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
+                                  const BwdTcParams& bp, int d, int grid, cudaStream_t stream) {
+    if (d == 128) return launch_bwd_tc<128>(tq, tdo, tk, tv, p_dq, p_dkv, bp, grid, stream);
+    if (d == 64) return launch_bwd_tc<64>(tq, tdo, tk, tv, p_dq, p_dkv, bp, grid, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace relbias

@@ -54,6 +54,26 @@ cudaError_t launch_prefill_fp32(const float* q, const float* k, const float* v, 
                                 cudaStream_t stream);
 constexpr int kMaxBankC = 16;   // functions in a shared bank
 
+// Backward pass on the tcgen05 tensor cores (backward_sm100.cu), bf16 inputs, d in {64, 128}.
+// Scheduling, r, w, R, window, scale and temperature come in a PrefillParams (nslots = 1,
+// HP = G; for the dK/dV kernel total_items counts (sequence, kv head, key tile)).
+struct BwdTcParams {
+    const __nv_bfloat16* o;     // [B, T, Hq, d] forward output
+    const __nv_bfloat16* dout;  // [B, T, Hq, d]
+    const float* lse;           // [B, Hq, T] forward log-sum-exp
+    float* dvec;                // [B, Hq, T] D_i = dout_i . o_i (written by the dQ kernel)
+    float* dq;                  // [B, T, Hq, d]
+    float* dr;                  // [B, T, Hq]
+    float* dk;                  // [B, T, Hkv, d]
+    float* dv;                  // [B, T, Hkv, d]
+    float* dw;                  // [Hq, R], zeroed by the caller, accumulated atomically
+    float scale;
+};
+bool backward_tc_supported(int d, int R);
+cudaError_t launch_backward_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
+                                  const BwdTcParams& bp, int d, int grid, cudaStream_t stream);
+
 // Backward pass on CUDA cores (backward_fp32.cu): dq [B,T,Hq,d], dk/dv [B,T,Hkv,d], dr
 // [B,T,Hq], dw [Hq,R] (zeroed here, then accumulated), all fp32; q, k, v, o, dout in
 // bf16 (bf16 == true) or fp32; dvec [B,Hq,T] scratch for D_i = dout_i . o_i.

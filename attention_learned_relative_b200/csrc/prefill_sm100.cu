@@ -547,11 +547,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int cp = base & (NCOPY - 1);
                     if constexpr (NCOPY == 0) {
                         if (row_ok) {
-                            add_bias_curves(s, curve_row, delta0 + t - (kBN - 1), p.R, rs);
-                            // The next tile's run (128 distances further) into L2 meanwhile.
-                            const int dn = delta0 + t + 1;   // its first distance
-                            if (tt + 1 < ntiles && dn < p.R)
-                                for (int k = 0; k < kBN; k += 32) prefetch_l2(curve_row + dn + k);
+                            const int dlo = delta0 + t - (kBN - 1);
+                            add_bias_curves(s, curve_row, dlo, p.R, rs);
+                            // The next key tile's run (the 128 distances below this one's)
+                            // into L2 meanwhile; addresses clamped into the row's curve.
+                            if (tt + 1 < ntiles && dlo > 0) {
+#pragma unroll
+                                for (int k = 0; k < kBN; k += 32)
+                                    prefetch_l2(curve_row + min(max(dlo - kBN + k, 0), p.R - 1));
+                            }
                         }
                     } else {
                         add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);

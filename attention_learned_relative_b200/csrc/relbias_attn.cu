@@ -18,6 +18,7 @@
 #include "prefill_fp32.cu"
 #include "prefill_sm100.cu"
 #include "backward_fp32.cu"
+#include "backward_sm100.cu"
 
 namespace relbias {
 namespace {
@@ -508,6 +509,65 @@ extern "C" int relbias_attn_decode_paged(const void* q, const void* k_pages, con
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "paged decode launch");
 }
 
+namespace {
+// The backward pass on the tcgen05 tensor cores: the dQ / dr kernel, then the
+// dK / dV / dw kernel (which reads the D_i = dout_i . o_i the first one writes).
+int bwd_tc_impl(const void* q, const void* k, const void* v, const float* r, const float* w, const void* o,
+                const float* lse, const void* dout, float* dq, float* dk, float* dv, float* dr, float* dw, int B,
+                int T, int Hq, int Hkv, int d, int window, int R, float scale, int temp_n0, float* dvec, int sms,
+                cudaStream_t st) {
+    int rc;
+    CUtensorMap tq, tdo, tk, tv;
+    if ((rc = make_map(&tq, q, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tdo, dout, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tk, k, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v, B, T, Hkv, d, 128)) != RELBIAS_OK) return rc;
+    PrefillParams p{};
+    p.r = r;
+    p.w = w;
+    p.B = B;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.nslots = 1;
+    p.HP = p.G;
+    p.window = window > 0 ? window : 0;
+    p.R = R;
+    p.n_qt = (T + 127) / 128;
+    p.q_off = 0;
+    p.kv_T = T;
+    p.contiguous = p.window > 0 ? 1 : 0;
+    p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
+    p.temp_n0 = temp_n0 > 1 ? temp_n0 : 0;
+    p.inv_log_n0 = temp_n0 > 1 ? static_cast<float>(1.0 / std::log(static_cast<double>(temp_n0))) : 0.0f;
+    PrefillParams p_dq = p, p_dkv = p;
+    const long long n_dq = static_cast<long long>(p.n_qt) * B * Hq;
+    const long long n_dkv = static_cast<long long>(p.n_qt) * B * Hkv;
+    if (n_dq > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", n_dq);
+    p_dq.total_items = static_cast<int>(n_dq);
+    p_dkv.total_items = static_cast<int>(n_dkv);
+    BwdTcParams bp{};
+    bp.o = static_cast<const __nv_bfloat16*>(o);
+    bp.dout = static_cast<const __nv_bfloat16*>(dout);
+    bp.lse = lse;
+    bp.dvec = dvec;
+    bp.dq = dq;
+    bp.dr = dr;
+    bp.dk = dk;
+    bp.dv = dv;
+    bp.dw = dw;
+    bp.scale = scale;
+    if (R > 0) {
+        const cudaError_t e = cudaMemsetAsync(dw, 0, static_cast<size_t>(Hq) * R * sizeof(float), st);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing dw");
+    }
+    const cudaError_t e = launch_backward_sm100(tq, tdo, tk, tv, p_dq, p_dkv, bp, d, sms, st);
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "backward launch");
+}
+}  // namespace
+
 extern "C" size_t relbias_attn_bwd_workspace_size(int B, int T, int Hq) {
     if (B < 0 || T < 0 || Hq < 1) return 0;
     const size_t n = static_cast<size_t>(B) * Hq * T * sizeof(float);
@@ -537,9 +597,17 @@ extern "C" int relbias_attn_bwd(const void* q, const void* k, const void* v, con
     if (ws_bytes < relbias_attn_bwd_workspace_size(B, T, Hq))
         return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes,
                     relbias_attn_bwd_workspace_size(B, T, Hq));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == RELBIAS_BF16 && (d == 64 || d == 128) && backward_tc_supported(d, R)) {
+        DeviceInfo dev;
+        if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+        if (dev.major == 10 && dev.minor == 0) return bwd_tc_impl(q, k, v, r, w, o, lse, dout, dq, dk, dv, dr, dw,
+                                                                  B, T, Hq, Hkv, d, window, R, scale, temp_n0,
+                                                                  static_cast<float*>(workspace), dev.sms, st);
+    }
     const cudaError_t e = launch_backward(dtype == RELBIAS_BF16, d, q, k, v, r, w, o, lse, dout, dq, dk, dv, dr, dw,
                                           static_cast<float*>(workspace), B, T, Hq, Hkv, window > 0 ? window : 0, R,
-                                          scale, temp_n0 > 1 ? temp_n0 : 0, static_cast<cudaStream_t>(stream));
+                                          scale, temp_n0 > 1 ? temp_n0 : 0, st);
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "backward launch");
 }
 

@@ -416,19 +416,22 @@ def roofline_of(wl, ms_step, peaks, peaks_kind):
                           "algorithmic_bytes_per_launch": per_step}
     per_step = wl.masked_flops()
     achieved = per_step / (ms_step * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    if wl.dtype != "bf16" or wl.backward:
-        # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
-        peak = 148 * 128 * 2 * 1.965e9 / 1e12
-    tensor = wl.dtype == "bf16" and not wl.backward
+    # bf16 runs on the tcgen05 tensor cores (the backward too, for d in {64, 128});
+    # fp32 on CUDA cores: 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz.
+    tensor = wl.dtype == "bf16" and (not wl.backward or wl.d in (64, 128))
+    peak = float(peaks["bf16_tflops"]) if tensor else 148 * 128 * 2 * 1.965e9 / 1e12
+    if wl.backward:
+        kernel = "bwd_dq_sm100_kernel + bwd_dkv_sm100_kernel" if tensor else "bwd_dq_kernel + bwd_dkv_kernel"
+    elif wl.dtype == "bf16":
+        kernel = "bank_rows_kernel + prefill_bf16_sm100_kernel" if wl.bank_C > 0 else "prefill_bf16_sm100_kernel"
+    else:
+        kernel = "prefill_fp32_kernel"
     return per_step, {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                       "frac": achieved / peak, "traffic": traffic,
                       "peak_source": (peaks_kind + " bf16_tflops (burst)") if tensor
                       else "fp32 FMA units x max clock",
                       "frac_of_datasheet_2250": achieved / 2250.0,
-                      "kernel": "bwd_dq_kernel + bwd_dkv_kernel" if wl.backward
-                      else ("bank_rows_kernel + prefill_bf16_sm100_kernel" if wl.bank_C > 0 and wl.dtype == "bf16"
-                            else ("prefill_bf16_sm100_kernel" if wl.dtype == "bf16" else "prefill_fp32_kernel")),
+                      "kernel": kernel,
                       "algorithmic_flops_per_launch": per_step}
 
 

@@ -1,6 +1,8 @@
 """GPU parity of the backward pass (relbias_attn_bwd) against the fp64 oracle's
 gradients (oracle_attn_bwd, itself pinned by finite differences of the forward).
 
+bf16 inputs with d in {64, 128} run on the tcgen05 kernels (backward_sm100.cu), fp32
+and other head sizes on the CUDA-core kernels (backward_fp32.cu).
 The kernel gets O and LSE from the oracle's forward (stored in the kernel's dtype),
 as a training step would get them from the forward pass.  Tolerance, relative to the
 largest reference gradient of each tensor: 1e-4 for fp32 (fp32 sums of up to a few
@@ -57,6 +59,10 @@ CASES = [
     (torch.float32, 1, 64, 2, 1, 64, 0, 0, 0),          # R = 0: no bias, no dw
     (torch.bfloat16, 1, 256, 8, 2, 128, 0, 128, 0),
     (torch.bfloat16, 1, 1024, 8, 2, 128, 512, 512, 0),  # the local-layer shape over 32 tiles
+    (torch.bfloat16, 1, 300, 6, 2, 64, 0, 100, 0),      # d = 64, group 3, ragged last tile
+    (torch.bfloat16, 2, 200, 4, 4, 128, 0, 300, 100),   # group 1, R beyond T, temperature
+    (torch.bfloat16, 1, 129, 4, 2, 128, 64, 32, 0),     # one tile plus one row, window < tile
+    (torch.bfloat16, 1, 1024, 32, 4, 128, 512, 512, 0), # the local layer's 32 / 4 head layout
 ]
 
 
@@ -89,12 +95,13 @@ def test_backward_after_the_bf16_forward():
     _check(g, ref, 2e-2, "backward after forward")
 
 
-def test_backward_is_deterministic_except_dw():
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_is_deterministic_except_dw(dtype):
     """dq, dk, dv and dr are written without atomics: bitwise repeatable."""
-    x = _inputs(torch.float32, 1, 200, 4, 2, 64, 64, seed=11)
+    x = _inputs(dtype, 1, 200, 4, 2, 64, 64, seed=11)
     o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["r"].cpu(), x["w"].cpu(), 0, 64,
                                     0.125)
-    o = torch.as_tensor(o_ref).float().cuda()
+    o = torch.as_tensor(o_ref).to(dtype).cuda()
     lse = torch.as_tensor(lse_ref).float().cuda()
     g1 = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], 0, 64, 0.125)
     g2 = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], 0, 64, 0.125)
