@@ -34,6 +34,14 @@ struct PrefillParams {
     // curve_stride floats written by launch_bank_rows; r and w are then unused.
     const float* curves;
     int curve_stride;
+    // Paged chunks (paged != 0): K/V live in a page pool [num_pages, page_size, Hkv, d],
+    // sequence b's logical block k in page block_table[b * max_pages + k]; sequence b's
+    // chunk has q_lens[b] rows (<= T) at positions q_offs[b] ... (both on the device).
+    int paged;
+    const int* block_table;
+    const int* q_offs;
+    const int* q_lens;
+    int page_size, max_pages, num_pages;
 };
 int prefill_bf16_table_copies(int d, int R);   // 0 if R does not fit shared memory
 // Shared-bank curves of every prefill row: [B, T, Hq] rows of prefill_bank_curve_stride(R)

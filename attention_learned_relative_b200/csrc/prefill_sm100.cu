@@ -142,6 +142,87 @@ __device__ __forceinline__ void kv_range(const PrefillParams& p, int i0, int& j_
     ntiles = (j_last - j_first) / kBN + 1;
 }
 
+// One 128-key tile of K or V from a page pool: two 64-row boxes, each inside one page
+// (page_size is a multiple of 64).  Rows in a block past the table, or in a page index
+// outside the pool, read zeros (TMA fills coordinates outside the tensor); the latter is
+// reported when the row is one the chunk attends.
+template <int D>
+__device__ __forceinline__ void load_kv_paged(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                              const PrefillParams& p, const Item& it, int j0, int kv_end) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int row = j0 + 64 * half;
+        const int blk = row / p.page_size;
+        int page = -1, prow = 0;
+        if (blk < p.max_pages) {
+            page = __ldg(p.block_table + static_cast<size_t>(it.b) * p.max_pages + blk);
+            prow = row - blk * p.page_size;
+            if ((page < 0 || page >= p.num_pages) && row < kv_end) atomicOr(&g_status, kStatusBadLength);
+        }
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_4d(dst + bx * kBM * 128 + half * 64 * 128, map, bar, bx * 64, it.g, prow, page);
+    }
+}
+
+// Zero rows [first, 128) of a 128-row tile (D/64 boxes of 128-byte rows; the swizzle
+// permutes chunks within a row, so whole rows are swizzle-free), by the 32 lanes of a
+// warp, then order the writes before the tensor cores' reads of the tile.
+template <int D>
+__device__ __forceinline__ void zero_rows(uint8_t* tile, int first, int lane) {
+    for (int x = lane; x < (kBM - first) * (D / 64) * 8; x += 32) {
+        const int row = first + x / ((D / 64) * 8);
+        const int rem = x % ((D / 64) * 8);
+        *reinterpret_cast<uint4*>(tile + (rem >> 3) * kBM * 128 + row * 128 + (rem & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_shared();
+    __syncwarp();
+}
+
+// Position of an item's first query row and its number of valid rows.  A chunk of
+// a paged cache reads its sequence's offset and length from the device arrays
+// (clamped into range and reported, when they are not).
+template <bool PAGED>
+__device__ __forceinline__ void item_rows(const PrefillParams& p, const Item& it, int& qo, int& nrows, int& kv_end) {
+    const int i0 = it.qt * kBM;
+    if constexpr (PAGED) {
+        int off = __ldg(p.q_offs + it.b), len = __ldg(p.q_lens + it.b);
+        const int cap = p.max_pages * p.page_size;
+        if (off < 0 || len < 0 || len > p.T || static_cast<long long>(off) + len > cap) {
+            atomicOr(&g_status, kStatusBadLength);
+            off = min(max(off, 0), cap);
+            len = min(max(len, 0), min(p.T, cap - off));
+        }
+        qo = off;
+        nrows = min(kBM, len - i0);
+        kv_end = off + len;
+    } else {
+        qo = p.q_off;
+        nrows = min(kBM, p.T - i0);
+        kv_end = p.q_off + p.T;
+    }
+}
+
+// Key tiles of an item.  A paged item with no valid rows visits one tile (its outputs
+// are not written), so every role walks the same tile stream.
+template <bool PAGED>
+__device__ __forceinline__ void item_kv_range(const PrefillParams& p, int i0, int qo, int nrows, int& j_first,
+                                              int& ntiles) {
+    if constexpr (PAGED) {
+        if (nrows <= 0) {
+            j_first = 0;
+            ntiles = 1;
+            return;
+        }
+        const int a0 = qo + i0;
+        const int lo = p.window > 0 ? max(0, a0 - p.window + 1) : 0;
+        j_first = (lo / kBN) * kBN;
+        ntiles = (a0 + nrows - 1) / kBN - j_first / kBN + 1;
+    } else {
+        kv_range(p, i0, j_first, ntiles);
+    }
+}
+
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 // The four softmax warps of a slot meet: each arrives once (after its own shared-memory
@@ -260,8 +341,10 @@ __device__ __forceinline__ void add_bias_curves(float (&s)[kBN], const float* ro
 }
 
 // NCOPY == 0: the shared-bank form, with each row's bias curve read from global
-// memory (no staged table).
-template <int D, int NCOPY>
+// memory (no staged table).  PAGED: K and V come from a page pool through a block
+// table, each 128-key tile as two 64-row boxes (the pool's tensor maps have 64-row
+// boxes), and every sequence has its own chunk offset and length.
+template <int D, int NCOPY, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -329,8 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int item_it = 0; ok && item_it < nitems; ++item_it) {
                 const Item it = item_at(p, item_it);
                 const int i0 = it.qt * kBM;
-                int j_first, ntiles;
-                kv_range(p, i0, j_first, ntiles);
+                int qo, nrows, kv_end, j_first, ntiles;
+                item_rows<PAGED>(p, it, qo, nrows, kv_end);
+                item_kv_range<PAGED>(p, i0, qo, nrows, j_first, ntiles);
                 const int h0 = it.g * p.G + it.hp * p.nslots;
                 for (int s = 0; ok && s < p.nslots; ++s) {
                     if (item_it > 0 && !(ok = warp_all(mbar_wait(&bars->q_empty[s], (item_it - 1) & 1, abort_flag))))
@@ -358,17 +442,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = warp_all(mbar_wait(&bars->k_empty[st], ph ^ 1, abort_flag)))) break;
                     if (leader) {
                         mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
-                        for (int bx = 0; bx < D / 64; ++bx)
-                            tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st],
-                                        bx * 64, it.g, j0, it.b);
+                        if constexpr (PAGED) {
+                            load_kv_paged<D>(smem + L::kK + st * L::kTile, &tm_k, &bars->k_full[st], p, it, j0, kv_end);
+                        } else {
+                            for (int bx = 0; bx < D / 64; ++bx)
+                                tma_load_4d(smem + L::kK + st * L::kTile + bx * L::kBox, &tm_k, &bars->k_full[st],
+                                            bx * 64, it.g, j0, it.b);
+                        }
                     }
                     ++nk;
                     if (!(ok = warp_all(mbar_wait(&bars->v_empty[st], ph ^ 1, abort_flag)))) break;
                     if (leader) {
                         mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
-                        for (int bx = 0; bx < D / 64; ++bx)
-                            tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st],
-                                        bx * 64, it.g, j0, it.b);
+                        if constexpr (PAGED) {
+                            load_kv_paged<D>(smem + L::kV + st * L::kTile, &tm_v, &bars->v_full[st], p, it, j0, kv_end);
+                        } else {
+                            for (int bx = 0; bx < D / 64; ++bx)
+                                tma_load_4d(smem + L::kV + st * L::kTile + bx * L::kBox, &tm_v, &bars->v_full[st],
+                                            bx * 64, it.g, j0, it.b);
+                        }
                     }
                     ++nv;
                 }
@@ -393,8 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nitems = items_of_cta(p);
             for (int item_it = 0; ok && item_it < nitems; ++item_it) {
                 const Item it = item_at(p, item_it);
-                int j_first, ntiles;
-                kv_range(p, it.qt * kBM, j_first, ntiles);
+                int qo, nrows, kv_end, j_first, ntiles;
+                item_rows<PAGED>(p, it, qo, nrows, kv_end);
+                item_kv_range<PAGED>(p, it.qt * kBM, qo, nrows, j_first, ntiles);
                 int prev_st = 0;
                 for (int t = 0; t < ntiles; ++t, ++kv_it) {
                     const int st = kv_it & 1;
@@ -424,6 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (leader) umma_commit(&bars->k_empty[st]);
                     if (!(ok = warp_all(mbar_wait(&bars->v_full[st], ph, abort_flag)))) break;
+                    if constexpr (PAGED) {
+                        // Cache rows at or past the sequence's end may hold anything, and a
+                        // NaN times a zero weight is NaN: zero those rows of the V tile before
+                        // the first PV that reads it (both slots' PVs come after).
+                        const int dead = kv_end - (j_first + t * kBN);
+                        if (dead < kBN) zero_rows<D>(smem + L::kV + st * L::kTile, max(dead, 0), lane);
+                    }
                     if (!(ok = warp_all(mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag)))) break;
                     ++pcnt[0];
                     tc_fence_after();
@@ -465,8 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item_it = 0; ok && item_it < nitems; ++item_it) {
             const Item it = item_at(p, item_it);
             const int i0 = it.qt * kBM;
-            int j_first, ntiles;
-            kv_range(p, i0, j_first, ntiles);
+            int qo, nrows, kv_end, j_first, ntiles;
+            item_rows<PAGED>(p, it, qo, nrows, kv_end);
+            item_kv_range<PAGED>(p, i0, qo, nrows, j_first, ntiles);
             const int h = it.g * p.G + it.hp * p.nslots + slot;
 
             // This head's reversed distance table, NCOPY shifted copies, staged when the
@@ -500,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 
             const int i = i0 + t;
-            const bool row_ok = i < p.T;
+            const bool row_ok = t < nrows;
             // Bias coefficient, in units of the unscaled logit: r_i / scale (rank-1 form), or
             // 1 / scale for the bank form, whose curve holds the whole bias.
             float rs = 0.0f;
@@ -509,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 rs = row_ok ? p.inv_scale : 0.0f;
                 curve_row = p.curves +
                             (static_cast<size_t>(it.b) * p.T + (row_ok ? i : 0)) * p.Hq * p.curve_stride +
-                            static_cast<size_t>(h) * p.curve_stride + (7 - ((p.q_off + i) & 7));
+                            static_cast<size_t>(h) * p.curve_stride + (7 - ((qo + i) & 7));
             } else {
                 rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale : 0.0f;
             }
@@ -521,14 +622,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // context length").
             float c1 = p.scale_log2;
             if (p.temp_n0 > 1) {
-                const int n = p.window > 0 ? min(p.q_off + i + 1, p.window) : p.q_off + i + 1;
+                const int n = p.window > 0 ? min(qo + i + 1, p.window) : qo + i + 1;
                 if (n > p.temp_n0) c1 *= __logf(static_cast<float>(n)) * p.inv_log_n0;
             }
             const uint64_t c1x2 = f2_pack(c1, c1);
 
             for (int tt = 0; tt < ntiles; ++tt, ++tile_it) {
                 const int j0 = j_first + tt * kBN;
-                const int delta0 = p.q_off + i0 - j0;   // distance of (row t, key c) is delta0 + t - c
+                const int delta0 = qo + i0 - j0;   // distance of (row t, key c) is delta0 + t - c
                 ok = warp_all(mbar_wait(&bars->s_full[slot], tile_it & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
@@ -682,10 +783,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, int NCOPY>
+template <int D, int NCOPY, bool PAGED = false>
 cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const PrefillParams& p, int smem, int grid, cudaStream_t stream) {
-    auto kern = prefill_bf16_sm100_kernel<D, NCOPY>;
+    auto kern = prefill_bf16_sm100_kernel<D, NCOPY, PAGED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
@@ -779,6 +880,16 @@ cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& 
     const int nc = prefill_bf16_table_copies(d, p.R);
     const int smem = prefill_bf16_smem_bytes(d, p.R);
     if (nc == 0 || smem < 0) return cudaErrorInvalidValue;
+    if (p.paged) {
+        if (d == 128) {
+            if (nc == 4) return launch_variant<128, 4, true>(tq, tk, tv, p, smem, grid, stream);
+            if (nc == 2) return launch_variant<128, 2, true>(tq, tk, tv, p, smem, grid, stream);
+            return launch_variant<128, 1, true>(tq, tk, tv, p, smem, grid, stream);
+        }
+        if (nc == 4) return launch_variant<64, 4, true>(tq, tk, tv, p, smem, grid, stream);
+        if (nc == 2) return launch_variant<64, 2, true>(tq, tk, tv, p, smem, grid, stream);
+        return launch_variant<64, 1, true>(tq, tk, tv, p, smem, grid, stream);
+    }
     if (d == 128) {
         if (nc == 4) return launch_variant<128, 4>(tq, tk, tv, p, smem, grid, stream);
         if (nc == 2) return launch_variant<128, 2>(tq, tk, tv, p, smem, grid, stream);

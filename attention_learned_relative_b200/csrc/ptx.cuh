@@ -140,6 +140,11 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c
                  "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
+// Order this thread's generic-proxy shared-memory writes before later async-proxy
+// (TMA, tcgen05.mma) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 // Pull the 128-byte line holding `p` into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));

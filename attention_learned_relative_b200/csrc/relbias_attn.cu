@@ -238,6 +238,78 @@ extern "C" int relbias_attn_fwd_chunk(const void* q, const void* k, const void* 
                     stream);
 }
 
+// Chunked prefill against a paged cache: every sequence's chunk at its own offset.
+extern "C" int relbias_attn_fwd_chunk_paged(const void* q, const void* k_pages, const void* v_pages,
+                                            const int* block_table, const int* q_offs, const int* q_lens,
+                                            const float* r, const float* w, void* o, float* lse, int B, int T,
+                                            int num_pages, int page_size, int max_pages, int Hq, int Hkv, int d,
+                                            int window, int R, float scale, int temp_n0, int dtype, void* stream) {
+    t_err.clear();
+    int rc = check_common(B, T, Hq, Hkv, d, R, scale, w);
+    if (rc != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0 || T == 0) return RELBIAS_OK;
+    if (num_pages < 1 || max_pages < 1)
+        return fail(RELBIAS_ERR_ARG, "num_pages (%d) and max_pages (%d) must be >= 1", num_pages, max_pages);
+    if (page_size < 64 || page_size % 64 != 0)
+        return fail(RELBIAS_ERR_ARG, "page_size (%d) must be a positive multiple of 64", page_size);
+    if (!q || !k_pages || !v_pages || !block_table || !q_offs || !q_lens || !r || !o)
+        return fail(RELBIAS_ERR_ARG, "q, k_pages, v_pages, block_table, q_offs, q_lens, r and o must not be null");
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o))
+        return fail(RELBIAS_ERR_ARG, "q, k_pages, v_pages and o must be 16-byte aligned");
+    if (!aligned4(r) || !aligned4(block_table) || !aligned4(q_offs) || !aligned4(q_lens) || (lse && !aligned4(lse)))
+        return fail(RELBIAS_ERR_ARG, "r, block_table, q_offs, q_lens and lse must be 4-byte aligned");
+    if (dtype != RELBIAS_BF16) return fail(RELBIAS_ERR_UNSUPPORTED, "the paged chunked prefill is bf16 only");
+    if (d != 64 && d != 128) return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill supports d in {64, 128}, got %d", d);
+    if (R > 2048 || prefill_bf16_table_copies(d, R) == 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill stages R <= 2048 table entries, got %d", R);
+    DeviceInfo dev;
+    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "bf16 prefill needs compute capability 10.0 (sm_100a), found %d.%d",
+                    dev.major, dev.minor);
+    CUtensorMap tq, tk, tv;
+    if ((rc = make_map(&tq, q, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tk, k_pages, num_pages, page_size, Hkv, d, 64)) != RELBIAS_OK) return rc;
+    if ((rc = make_map(&tv, v_pages, num_pages, page_size, Hkv, d, 64)) != RELBIAS_OK) return rc;
+    PrefillParams p{};
+    p.r = r;
+    p.w = w;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.nslots = (p.G % 2 == 0) ? 2 : 1;
+    p.HP = p.G / p.nslots;
+    p.window = window > 0 ? window : 0;
+    p.R = R;
+    p.n_qt = (T + 127) / 128;
+    p.q_off = 0;
+    p.kv_T = T;
+    const long long items = static_cast<long long>(p.n_qt) * B * Hkv * p.HP;
+    if (items > INT32_MAX) return fail(RELBIAS_ERR_UNSUPPORTED, "too many work items (%lld)", items);
+    p.total_items = static_cast<int>(items);
+    p.contiguous = p.window > 0 ? 1 : 0;
+    p.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
+    p.scale_log2 = scale * kLog2e;
+    p.inv_scale = 1.0f / scale;
+    p.temp_n0 = temp_n0 > 1 ? temp_n0 : 0;
+    p.inv_log_n0 = temp_n0 > 1 ? static_cast<float>(1.0 / std::log(static_cast<double>(temp_n0))) : 0.0f;
+    p.paged = 1;
+    p.block_table = block_table;
+    p.q_offs = q_offs;
+    p.q_lens = q_lens;
+    p.page_size = page_size;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    const int grid = static_cast<int>(std::min<long long>(items, dev.sms));
+    const cudaError_t e = launch_prefill_bf16_sm100(tq, tk, tv, p, d, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "paged chunked prefill launch");
+}
+
 namespace relbias {
 namespace {
 int check_bank(int C, int proj_heads, int Hq) {

@@ -35,6 +35,7 @@ SIGNATURES = {
     "relbias_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "relbias_attn_fwd_chunk": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                     _I, _VP]),
+    "relbias_attn_fwd_chunk_paged": (_I, [_VP] * 10 + [_I] * 10 + [_F, _I, _I, _VP]),
     "relbias_attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "relbias_attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP,
                                  _SZ, _VP]),
@@ -163,6 +164,42 @@ def attn_fwd_chunk(q, k, v, r, w, q_off: int, window: int, R: int, scale: float 
     rc = lib().relbias_attn_fwd_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(r), _ptr(w), _ptr(out), _ptr(lse),
                                       B, T, int(q_off), kv_T, Hq, Hkv, d, int(window), int(R), float(scale),
                                       int(temp_n0), _dtype_code(q), _stream_handle(stream, q.device))
+    _check(rc)
+    return out
+
+
+def attn_fwd_chunk_paged(q, k_pages, v_pages, block_table, q_offs, q_lens, r, w, window: int, R: int,
+                         scale: float | None = None, out=None, lse=None, stream=None, temp_n0: int = 0):
+    """Chunked prefill against a paged cache.  q [B,T,Hq,d] bf16 (sequence b's chunk is
+    its first q_lens[b] rows, at positions q_offs[b] ...), k_pages/v_pages
+    [num_pages,page_size,Hkv,d] bf16, block_table [B,max_pages] int32, q_offs/q_lens [B]
+    int32, r [B,T,Hq] fp32, w [Hq,R] fp32.  Returns o [B,T,Hq,d]; rows at or past
+    q_lens[b] are left as they were in `out` (allocated, uninitialised, if None)."""
+    _need(q.dim() == 4 and k_pages.dim() == 4 and v_pages.shape == k_pages.shape,
+          "q [B,T,Hq,d], pages [num_pages,page_size,Hkv,d]")
+    B, T, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_pages.shape
+    _need(dk == d, "page head dim %d != q head dim %d" % (dk, d))
+    _need(q.dtype == k_pages.dtype == v_pages.dtype, "q and pages must share a dtype")
+    _need(block_table.dim() == 2 and block_table.shape[0] == B and block_table.dtype == torch.int32,
+          "block_table must be int32 [B, max_pages]")
+    for name, t_ in (("q_offs", q_offs), ("q_lens", q_lens)):
+        _need(t_.shape == (B,) and t_.dtype == torch.int32, "%s must be int32 [B]" % name)
+    _need(r.shape == (B, T, Hq) and r.dtype == torch.float32, "r must be fp32 [B,T,Hq]")
+    _need(w is None or (w.shape == (Hq, R) and w.dtype == torch.float32), "w must be fp32 [Hq,R]")
+    for t_ in (q, k_pages, v_pages, block_table, q_offs, q_lens, r, w, out, lse):
+        _need(t_ is None or (t_.is_cuda and t_.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out.shape == q.shape and out.dtype == q.dtype, "out must match q")
+    _need(lse is None or (lse.shape == (B, Hq, T) and lse.dtype == torch.float32), "lse must be fp32 [B,Hq,T]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_fwd_chunk_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(q_offs),
+                                            _ptr(q_lens), _ptr(r), _ptr(w), _ptr(out), _ptr(lse), B, T, num_pages,
+                                            page_size, block_table.shape[1], Hq, Hkv, d, int(window), int(R),
+                                            float(scale), int(temp_n0), _dtype_code(q),
+                                            _stream_handle(stream, q.device))
     _check(rc)
     return out
 

@@ -127,6 +127,39 @@ RELBIAS_API int relbias_attn_fwd_chunk(const void* q, const void* k, const void*
                      int dtype, void* stream);
 
 /*
+ * Chunked prefill against a paged, variable-length cache: the paged KV cache and
+ * variable sequence lengths the essay ("Thinking Machines dropped RoPE", closing
+ * section on kernel cost) lists among what a production attention kernel covers.
+ * Sequence b's chunk has q_lens[b] rows (0 <= q_lens[b] <= T) at positions
+ * q_offs[b] ... q_offs[b]+q_lens[b]-1; its keys and values, the prefix and the
+ * chunk's own rows, are cache rows 0 ... q_offs[b]+q_lens[b]-1, where cache row t of
+ * sequence b is row t % page_size of page block_table[b][t / page_size].  Same
+ * computation as relbias_attn_fwd_chunk for each sequence.
+ *
+ *   q, o     [B, T, Hq, d]          bf16   rows >= q_lens[b] are neither read for a
+ *                                          result nor written (o, lse keep their contents)
+ *   r        [B, T, Hq]             fp32
+ *   lse      [B, Hq, T]             fp32   may be NULL
+ *   k_pages, v_pages [num_pages, page_size, Hkv, d]   bf16, the page pool
+ *   block_table      [B, max_pages]  int32  (device)
+ *   q_offs, q_lens   [B]             int32  (device, read by the kernel)
+ *   page_size a positive multiple of 64; bf16 only, d in {64, 128}, R <= 2048.
+ *   An offset or length out of range (q_offs[b] + q_lens[b] > max_pages * page_size,
+ *   or q_lens[b] > T) is clamped into range, and a page index outside the pool reads
+ *   zeros; either sets RELBIAS_STATUS_BAD_LENGTH.  Cache rows past a sequence's end
+ *   may hold anything (they are never attended, and their values never reach a
+ *   product).
+ */
+RELBIAS_API int relbias_attn_fwd_chunk_paged(const void* q, const void* k_pages, const void* v_pages,
+                        const int* block_table, const int* q_offs, const int* q_lens,
+                        const float* r, const float* w,
+                        void* o, float* lse,
+                        int B, int T, int num_pages, int page_size, int max_pages,
+                        int Hq, int Hkv, int d,
+                        int window, int R, float scale, int temp_n0,
+                        int dtype, void* stream);
+
+/*
  * Decode: one new query per sequence at position n_ctx-1 against a key/value
  * cache of n_ctx rows whose last row already holds that query's own key and
  * value (the 1,048,576-token context of the archdiff.com model card, "Context").

@@ -314,3 +314,38 @@ def test_noalloc_reports_argument_errors_like_the_regular_decode(lib, kw):
 def test_noalloc_empty_batch(lib):
     assert _dec_noalloc(lib, B=0) == ops.RELBIAS_OK
     assert _dec_noalloc(lib, B=0, q=None, o=None) == ops.RELBIAS_OK
+
+
+def _chunk_paged(lib, **kw):
+    a = dict(q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, qo=FAKE, ql=FAKE, r=FAKE, w=FAKE, o=FAKE, lse=None, B=2, T=100,
+             num_pages=8, page_size=128, max_pages=4, Hq=8, Hkv=2, d=128, window=0, R=64, scale=0.1, temp_n0=0,
+             dtype=ops.RELBIAS_BF16)
+    a.update(kw)
+    return lib.relbias_attn_fwd_chunk_paged(a["q"], a["kp"], a["vp"], a["bt"], a["qo"], a["ql"], a["r"], a["w"],
+                                            a["o"], a["lse"], a["B"], a["T"], a["num_pages"], a["page_size"],
+                                            a["max_pages"], a["Hq"], a["Hkv"], a["d"], a["window"], a["R"],
+                                            a["scale"], a["temp_n0"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(page_size=96), ops.RELBIAS_ERR_ARG),           # not a multiple of 64
+    (dict(page_size=0), ops.RELBIAS_ERR_ARG),
+    (dict(num_pages=0), ops.RELBIAS_ERR_ARG),
+    (dict(max_pages=0), ops.RELBIAS_ERR_ARG),
+    (dict(bt=None), ops.RELBIAS_ERR_ARG),
+    (dict(qo=None), ops.RELBIAS_ERR_ARG),
+    (dict(ql=FAKE + 2), ops.RELBIAS_ERR_ARG),            # misaligned
+    (dict(kp=FAKE + 8), ops.RELBIAS_ERR_ARG),
+    (dict(Hq=9), ops.RELBIAS_ERR_ARG),
+    (dict(dtype=ops.RELBIAS_FP32), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(d=96), ops.RELBIAS_ERR_UNSUPPORTED),
+    (dict(R=4096), ops.RELBIAS_ERR_UNSUPPORTED),
+])
+def test_chunk_paged_rejects_on_host(lib, kw, code):
+    assert _chunk_paged(lib, **kw) == code
+    assert ops.last_error() != ""
+
+
+def test_chunk_paged_empty_is_a_no_op(lib):
+    assert _chunk_paged(lib, B=0) == ops.RELBIAS_OK
+    assert _chunk_paged(lib, T=0) == ops.RELBIAS_OK
