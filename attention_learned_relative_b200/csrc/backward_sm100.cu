@@ -84,6 +84,41 @@ struct TileCursor {
     __device__ __forceinline__ int j0() const { return j_first + t * kBN; }
 };
 
+// D_i = dO_i . O_i for every row (b, i, h), into dvec [B, Hq, T]: one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout, float* __restrict__ dvec,
+                                                       int B, int T, int Hq) {
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // (b * T + i) * Hq + h
+    const int lane = threadIdx.x & 31;
+    if (row >= static_cast<long long>(B) * T * Hq) return;
+    float acc = 0.0f;
+#pragma unroll
+    for (int u = lane * 2; u < D; u += 64) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + row * D + u));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + row * D + u));
+        acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        const int h = static_cast<int>(row % Hq);
+        const long long bi = row / Hq;
+        const int i = static_cast<int>(bi % T), b = static_cast<int>(bi / T);
+        dvec[(static_cast<size_t>(b) * Hq + h) * T + i] = acc;
+    }
+}
+
+// A dQ-kernel row's inputs: D_i, LSE_i (natural log) and r_i (zeros past T).
+__device__ __forceinline__ float3 bq_row_inputs(const PrefillParams& p, const BwdTcParams& bp, const Item& it, int t) {
+    const int i = it.qt * kBM + t;
+    if (i >= p.T) return make_float3(0.f, 0.f, 0.f);
+    const int h = it.g * p.G + it.hp;
+    const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + i;
+    return make_float3(__ldg(bp.dvec + hrow), __ldg(bp.lse + hrow),
+                       __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h));
+}
+
 template <int D, int NCOPY>
 __global__ void __launch_bounds__(kBqThreads, 1)
     bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -178,6 +213,12 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                         tma_load_4d(smem + L::kV + st * L::kTile + bx * kBM * 128, &tm_v, &bars->v_full[st],
                                     bx * 64, it.g, j0, it.b);
                     }
+                    // Warm L2 with the tile two ahead within the item (its stage frees late).
+                    if (t + 2 < ntiles)
+                        for (int bx = 0; bx < D / 64; ++bx) {
+                            tma_prefetch_l2_4d(&tm_k, bx * 64, it.g, j0 + 2 * kBN, it.b);
+                            tma_prefetch_l2_4d(&tm_v, bx * 64, it.g, j0 + 2 * kBN, it.b);
+                        }
                 }
                 ++nkv;
             }
@@ -255,12 +296,16 @@ __global__ void __launch_bounds__(kBqThreads, 1)
         uint32_t tab_phase = 0;
         int g = 0;
         bool ok = true;
+        // The row's D_i, LSE and bias feature are loaded one item ahead.
+        float3 nxt = nitems > 0 ? bq_row_inputs(p, bp, item_at(p, 0), t) : make_float3(0.f, 0.f, 0.f);
         for (int item_it = 0; ok && item_it < nitems; ++item_it) {
             const Item it = item_at(p, item_it);
             const int i0 = it.qt * kBM;
             int j_first, ntiles;
             kv_range(p, i0, j_first, ntiles);
             const int h = it.g * p.G + it.hp;
+            const float3 cur = nxt;
+            if (item_it + 1 < nitems) nxt = bq_row_inputs(p, bp, item_at(p, item_it + 1), t);
             if (h != staged_head) {
                 staged_head = h;
                 if (!(ok = tab_meet(&bars->tab_sync, tab_phase, abort_flag))) break;
@@ -276,33 +321,17 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             const bool row_ok = i < p.T;
             const size_t row = (static_cast<size_t>(it.b) * p.T + (row_ok ? i : 0)) * p.Hq + h;   // [B, T, Hq]
             const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + (row_ok ? i : 0);  // [B, Hq, T]
-            // D_i = dO_i . O_i, the row's log-sum-exp in log2 units, the logit scale with
-            // the context-length temperature, and the bias coefficient (log2 units).
-            float Di = 0.0f;
-            if (row_ok) {
-                const uint4* orow = reinterpret_cast<const uint4*>(bp.o + row * D);
-                const uint4* grow = reinterpret_cast<const uint4*>(bp.dout + row * D);
-#pragma unroll 4
-                for (int u = 0; u < D / 8; ++u) {
-                    const uint4 a = __ldg(orow + u), b = __ldg(grow + u);
-                    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
-                        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
-                        Di = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, Di));
-                    }
-                }
-                bp.dvec[hrow] = Di;
-            }
-            const float lse2 = row_ok ? __ldg(bp.lse + hrow) * 1.4426950408889634f : 0.0f;
+            // D_i (from the D kernel), the row's log-sum-exp in log2 units, the logit scale
+            // with the context-length temperature, and the bias coefficient (log2 units).
+            const float Di = cur.x;
+            const float lse2 = cur.y * 1.4426950408889634f;
             float tau = 1.0f;
             if (p.temp_n0 > 1) {
                 const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
                 if (n > p.temp_n0) tau = __logf(static_cast<float>(n)) * p.inv_log_n0;
             }
             const float c1 = p.scale_log2 * tau;
-            const float rb = row_ok ? __ldg(p.r + row) * p.inv_scale * c1 : 0.0f;   // bias, log2 units
+            const float rb = cur.z * p.inv_scale * c1;   // bias, log2 units
             const float ds_scale = tau * bp.scale;   // dS = tau * scale * dl, the dQ MMA's operand
             float dr_acc = 0.0f;                     // sum_j dl_j w[h, i-j]
 
@@ -480,6 +509,17 @@ __device__ __forceinline__ BkItem bk_item_at(const PrefillParams& p, int k) {
     return it;
 }
 
+// Query row qt * 128 + t of head (g * G + hl): its (r, LSE, D) (zeros past T).
+__device__ __forceinline__ float3 bk_col_inputs(const PrefillParams& p, const BwdTcParams& bp, const BkItem& it, int hl,
+                                                int qt, int t) {
+    const int i = qt * kBM + t;
+    if (i >= p.T) return make_float3(0.f, 0.f, 0.f);
+    const int h = it.g * p.G + hl;
+    const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + i;
+    return make_float3(__ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h), __ldg(bp.lse + hrow),
+                       __ldg(bp.dvec + hrow));
+}
+
 template <int D, int NCOPY>
 __global__ void __launch_bounds__(kBkThreads, 1)
     bwd_dkv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -636,6 +676,16 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         uint32_t col_phase = 0;
         int ns = 0;
         bool ok = true;
+        // Query row i0 + t's (r, LSE, D) for the next step, loaded one step ahead: steps
+        // run over (item, head of the group, query tile).
+        int s_item = 0, s_hl = 0, s_qt = 0;
+        bool s_valid = nitems > 0;
+        if (s_valid) {
+            int lo, hi;
+            q_range(p, bk_item_at(p, 0).kt, lo, hi);
+            s_qt = lo;
+        }
+        float3 nxt = s_valid ? bk_col_inputs(p, bp, bk_item_at(p, 0), 0, s_qt, t) : make_float3(0.f, 0.f, 0.f);
         for (int item_it = 0; ok && item_it < nitems; ++item_it) {
             const BkItem it = bk_item_at(p, item_it);
             const int k0 = it.kt * kBN;
@@ -659,21 +709,33 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 for (int qt = qt_lo; qt <= qt_hi; ++qt, ++ns) {
                     const int i0 = qt * kBM;
                     float4* cb = col + (ns & 1) * 2 * kBM;
+                    const float3 cur = nxt;
+                    {
+                        // The step after this one, and its inputs in flight meanwhile.
+                        if (++s_qt > qt_hi) {
+                            if (++s_hl >= p.G) {
+                                s_hl = 0;
+                                if (++s_item >= nitems) s_valid = false;
+                            }
+                            if (s_valid) {
+                                int lo, hi;
+                                q_range(p, bk_item_at(p, s_item).kt, lo, hi);
+                                s_qt = lo;
+                            }
+                        }
+                        if (s_valid) nxt = bk_col_inputs(p, bp, bk_item_at(p, s_item), s_hl, s_qt, t);
+                    }
                     {
                         // Column constants of query row i0 + t (this thread fills column t).
                         const int i = i0 + t;
-                        const bool row_ok = i < p.T;
-                        const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + (row_ok ? i : 0);
                         float tau = 1.0f;
                         if (p.temp_n0 > 1) {
                             const int n = p.window > 0 ? min(i + 1, p.window) : i + 1;
                             if (n > p.temp_n0) tau = __logf(static_cast<float>(n)) * p.inv_log_n0;
                         }
                         const float c1 = p.scale_log2 * tau;
-                        const float ri = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) : 0.0f;
-                        const float lse2 = row_ok ? __ldg(bp.lse + hrow) * 1.4426950408889634f : 0.0f;
-                        const float Di = row_ok ? bp.dvec[hrow] : 0.0f;
-                        cb[2 * t] = make_float4(c1, ri * p.inv_scale * c1, lse2, Di);
+                        const float ri = cur.x;
+                        cb[2 * t] = make_float4(c1, ri * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z);
                         cb[2 * t + 1] = make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
                     }
                     if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
@@ -797,6 +859,11 @@ template <int D>
 cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                           const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
                           const BwdTcParams& bp, int grid, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(p_dq.B) * p_dq.T * p_dq.Hq;
+    bwd_dvec_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(bp.o, bp.dout, bp.dvec, p_dq.B,
+                                                                                 p_dq.T, p_dq.Hq);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
     const int nc = bq_copies<D>(p_dq.R);
     cudaError_t e = nc == 4   ? launch_bq<D, 4>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)
                     : nc == 2 ? launch_bq<D, 2>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)

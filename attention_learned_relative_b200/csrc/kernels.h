@@ -49,7 +49,7 @@ int prefill_bf16_table_copies(int d, int R);   // 0 if R does not fit shared mem
 int prefill_bank_curve_stride(int R);
 cudaError_t launch_bank_rows(const float* rs, const float* proj, float* curves, int B, int T, int Hq, int q_off, int C,
                              int proj_heads, int R, cudaStream_t stream);
-int prefill_bf16_smem_bytes(int d, int R);
+int prefill_bf16_smem_bytes(int d, int R, int nc);
 cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream);
 

@@ -50,6 +50,9 @@ constexpr int kBN = 128;            // keys per tile
 constexpr int kStages = 2;          // K and V ring depth
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows by > 2^8
+// log2 units: a reference max may sit this far above a row's true running max (every
+// weight then stays >= 2^-64, far inside the range of fp32 and bf16).
+constexpr float kRefSlack = 64.0f;
 constexpr int kSoftmaxRegs = 216;
 constexpr int kOtherRegs = 72;
 constexpr int kMaxDynSmem = 232448;          // 227 KB per CTA on sm_100
@@ -224,6 +227,17 @@ __device__ __forceinline__ void item_kv_range(const PrefillParams& p, int i0, in
 }
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// The bias feature r[b, i, h] of this thread's row of an item (0 for rows past the
+// item's valid rows).
+template <bool PAGED>
+__device__ __forceinline__ float load_feature(const PrefillParams& p, const Item& it, int slot, int t) {
+    int qo, nrows, kv_end;
+    item_rows<PAGED>(p, it, qo, nrows, kv_end);
+    const int i = it.qt * kBM + t;
+    const int h = it.g * p.G + it.hp * p.nslots + slot;
+    return t < nrows ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) : 0.0f;
+}
 
 // The four softmax warps of a slot meet: each arrives once (after its own shared-memory
 // writes, which the arrival releases), then waits for the phase with a bounded wait.
@@ -473,6 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int n = max(0, nv - kStages); n < nv; ++n) mbar_drain_wait(&bars->v_full[n & 1], (n >> 1) & 1);
         } else if (warp == 9) {
             // -------------------------------------------------------- MMA issuer
+            // The key tiles of all this CTA's items form one stream g = 0, 1, ...; per tile
+            // the issue order is QK0(g) PV1(g-1) QK1(g) PV0(g), across item boundaries too:
+            // a slot's first QK of the next item follows its last PV directly, so the next
+            // item's first logits are computed while the softmax warps write the output.
             const bool leader = elect_one();
             const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
             const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
@@ -481,6 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
             int kv_it = 0;
             uint32_t pcnt[2] = {0, 0};
+            // Slot 1's PV of the previous tile (issued after the next tile's QK0).
+            bool prev = false, prev_first = false, prev_last = false;
+            int prev_st = 0;
             bool ok = true;
             const int nitems = items_of_cta(p);
             for (int item_it = 0; ok && item_it < nitems; ++item_it) {
@@ -488,32 +509,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int qo, nrows, kv_end, j_first, ntiles;
                 item_rows<PAGED>(p, it, qo, nrows, kv_end);
                 item_kv_range<PAGED>(p, it.qt * kBM, qo, nrows, j_first, ntiles);
-                int prev_st = 0;
                 for (int t = 0; t < ntiles; ++t, ++kv_it) {
                     const int st = kv_it & 1;
                     const uint32_t ph = (kv_it >> 1) & 1;
+                    const bool first = t == 0, last = t == ntiles - 1;
                     const uint32_t k_addr = smem_u32(smem + L::kK + st * L::kTile);
                     const uint32_t v_addr = smem_u32(smem + L::kV + st * L::kTile);
                     if (!(ok = warp_all(mbar_wait(&bars->k_full[st], ph, abort_flag)))) break;
-                    if (t == 0 && !(ok = warp_all(mbar_wait(&bars->q_full[0], item_it & 1, abort_flag)))) break;
+                    if (first && !(ok = warp_all(mbar_wait(&bars->q_full[0], item_it & 1, abort_flag)))) break;
                     tc_fence_after();
                     issue_qk<D>(leader, s_tm[0], q_addr[0], k_addr, idesc_qk);
                     if (leader) umma_commit(&bars->s_full[0]);
-                    if (leader && t == ntiles - 1) umma_commit(&bars->q_empty[0]);
+                    if (leader && last) umma_commit(&bars->q_empty[0]);
                     if (p.nslots == 2) {
-                        if (t > 0) {
+                        if (prev) {
                             if (!(ok = warp_all(mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag)))) break;
                             ++pcnt[1];
                             tc_fence_after();
                             issue_pv<D>(leader, o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile),
-                                        idesc_pv, t - 1 > 0);
+                                        idesc_pv, !prev_first);
                             if (leader) umma_commit(&bars->v_empty[prev_st]);
+                            if (leader && prev_last) umma_commit(&bars->o_final[1]);
                         }
-                        if (t == 0 && !(ok = warp_all(mbar_wait(&bars->q_full[1], item_it & 1, abort_flag)))) break;
+                        if (first && !(ok = warp_all(mbar_wait(&bars->q_full[1], item_it & 1, abort_flag)))) break;
                         tc_fence_after();
                         issue_qk<D>(leader, s_tm[1], q_addr[1], k_addr, idesc_qk);
                         if (leader) umma_commit(&bars->s_full[1]);
-                        if (leader && t == ntiles - 1) umma_commit(&bars->q_empty[1]);
+                        if (leader && last) umma_commit(&bars->q_empty[1]);
                     }
                     if (leader) umma_commit(&bars->k_empty[st]);
                     if (!(ok = warp_all(mbar_wait(&bars->v_full[st], ph, abort_flag)))) break;
@@ -527,19 +549,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = warp_all(mbar_wait(&bars->p_full[0], pcnt[0] & 1, abort_flag)))) break;
                     ++pcnt[0];
                     tc_fence_after();
-                    issue_pv<D>(leader, o_tm[0], s_tm[0], v_addr, idesc_pv, t > 0);
+                    issue_pv<D>(leader, o_tm[0], s_tm[0], v_addr, idesc_pv, !first);
                     if (leader && p.nslots == 1) umma_commit(&bars->v_empty[st]);
-                    if (leader && t == ntiles - 1) umma_commit(&bars->o_final[0]);
+                    if (leader && last) umma_commit(&bars->o_final[0]);
+                    prev = true;
                     prev_st = st;
+                    prev_first = first;
+                    prev_last = last;
                 }
-                if (ok && p.nslots == 2) {
-                    if (!(ok = warp_all(mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag)))) break;
-                    ++pcnt[1];
+            }
+            if (ok && p.nslots == 2 && prev) {
+                if ((ok = warp_all(mbar_wait(&bars->p_full[1], pcnt[1] & 1, abort_flag)))) {
                     tc_fence_after();
                     issue_pv<D>(leader, o_tm[1], s_tm[1], smem_u32(smem + L::kV + prev_st * L::kTile), idesc_pv,
-                                ntiles > 1);
+                                !prev_first);
                     if (leader) umma_commit(&bars->v_empty[prev_st]);
-                    if (leader) umma_commit(&bars->o_final[1]);
+                    if (leader && prev_last) umma_commit(&bars->o_final[1]);
                 }
             }
             // Drain: wait (bounded, regardless of abort) until every MMA issued has finished,
@@ -562,9 +587,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t tab_phase = 0;
         bool ok = slot < p.nslots;
         const int nitems = items_of_cta(p);
+        // The row's bias feature (rank-1 form) is loaded one item ahead, off the path
+        // between an item's last tile and the next item's first.
+        float r_next = 0.0f;
+        if (NCOPY > 0 && ok && nitems > 0) r_next = load_feature<PAGED>(p, item_at(p, 0), slot, t);
+        // The reference max an item's rows start from: the previous item's final running
+        // max of this thread's row (none for the first item).
+        float m_hint = -INFINITY;
         for (int item_it = 0; ok && item_it < nitems; ++item_it) {
             const Item it = item_at(p, item_it);
             const int i0 = it.qt * kBM;
+            const float r_cur = r_next;
+            if (NCOPY > 0 && item_it + 1 < nitems) r_next = load_feature<PAGED>(p, item_at(p, item_it + 1), slot, t);
             int qo, nrows, kv_end, j_first, ntiles;
             item_rows<PAGED>(p, it, qo, nrows, kv_end);
             item_kv_range<PAGED>(p, i0, qo, nrows, j_first, ntiles);
@@ -612,9 +646,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             (static_cast<size_t>(it.b) * p.T + (row_ok ? i : 0)) * p.Hq * p.curve_stride +
                             static_cast<size_t>(h) * p.curve_stride + (7 - ((qo + i) & 7));
             } else {
-                rs = row_ok ? __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * p.inv_scale : 0.0f;
+                rs = row_ok ? r_cur * p.inv_scale : 0.0f;
             }
-            float m_used = -INFINITY;   // running max, log2 units
+            // Running reference max (log2 units) and the largest tile max seen.  Every
+            // exponential is taken against m_used; m_used starts at the hint and is kept
+            // within [m_seen - kRefSlack, m_seen + kRescaleThreshold] once m_seen is finite.
+            float m_used = m_hint;
+            float m_seen = -INFINITY;
             uint64_t l2 = 0;            // running sum, two partial lanes (0.0f, 0.0f)
             // Logit scale of this row, log2 units, with the context-length temperature:
             // a row that sees n > temp_n0 keys has its logits (content and bias) scaled
@@ -633,99 +671,121 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = warp_all(mbar_wait(&bars->s_full[slot], tile_it & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t sr[kBN];
+                uint32_t pk[kBN / 2];
+                uint64_t acc[4];
+                // One pass: logits from S (still in tensor memory), bias and mask, then the
+                // exponentials against m_used with the tile's max found alongside.  A second
+                // pass runs only when the tile shows m_used to be off: its max more than
+                // 2^8 above it, or the first finite max of the item more than 2^64 below it
+                // (a hint far too high).  The row is then re-referenced at its running max.
+                for (int pass = 0;; ++pass) {
+                    uint32_t sr[kBN];
 #pragma unroll
-                for (int c = 0; c < kBN; c += 32) tmem_ld32(s_tm + c, sr + c);
-                tmem_ld_wait();
-                float s[kBN];
+                    for (int c = 0; c < kBN; c += 32) tmem_ld32(s_tm + c, sr + c);
+                    tmem_ld_wait();
+                    float s[kBN];
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+                    for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
 
-                if (delta0 - (kBN - 1) < p.R) {
-                    // Some key of this tile is closer than R: add r_i * w[h, i-j] (in units
-                    // of the unscaled logit; the table is zero outside [0, R)).
-                    const int base = cmax - delta0 - t;
-                    const int cp = base & (NCOPY - 1);
-                    if constexpr (NCOPY == 0) {
-                        if (row_ok) {
-                            const int dlo = delta0 + t - (kBN - 1);
-                            add_bias_curves(s, curve_row, dlo, p.R, rs);
-                            // The next key tile's run (the 128 distances below this one's)
-                            // into L2 meanwhile; addresses clamped into the row's curve.
-                            if (tt + 1 < ntiles && dlo > 0) {
+                    if (delta0 - (kBN - 1) < p.R) {
+                        // Some key of this tile is closer than R: add r_i * w[h, i-j] (in units
+                        // of the unscaled logit; the table is zero outside [0, R)).
+                        const int base = cmax - delta0 - t;
+                        const int cp = base & (NCOPY - 1);
+                        if constexpr (NCOPY == 0) {
+                            if (row_ok) {
+                                const int dlo = delta0 + t - (kBN - 1);
+                                add_bias_curves(s, curve_row, dlo, p.R, rs);
+                                // The next key tile's run (the 128 distances below this one's)
+                                // into L2 meanwhile; addresses clamped into the row's curve.
+                                if (pass == 0 && tt + 1 < ntiles && dlo > 0) {
 #pragma unroll
-                                for (int k = 0; k < kBN; k += 32)
-                                    prefetch_l2(curve_row + min(max(dlo - kBN + k, 0), p.R - 1));
+                                    for (int k = 0; k < kBN; k += 32)
+                                        prefetch_l2(curve_row + min(max(dlo - kBN + k, 0), p.R - 1));
+                                }
+                            }
+                        } else {
+                            add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
+                        }
+                    }
+                    if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
+                        // Key c is visible to row t iff lo <= c <= hi.  A 32-column chunk the
+                        // whole warp sees entirely is skipped (a warp-uniform branch); other
+                        // chunks pay per-element compares.
+                        const int hi = delta0 + t;
+                        const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
+                        const int t0 = t & ~31;
+                        const int hi_min = delta0 + t0;
+                        const int lo_max = p.window > 0 ? hi_min + 31 - p.window + 1 : INT_MIN;
+#pragma unroll
+                        for (int cc = 0; cc < kBN; cc += 32) {
+                            if (!(hi_min >= cc + 31 && lo_max <= cc)) {               // not all visible
+#pragma unroll
+                                for (int c = cc; c < cc + 32; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
                             }
                         }
-                    } else {
-                        add_bias<NCOPY>(s, wtab + cp * tstride + (base - cp), rs);
                     }
-                }
-                if (delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window)) {
-                    // Key c is visible to row t iff lo <= c <= hi.  A 32-column chunk the
-                    // whole warp sees entirely is skipped (a warp-uniform branch); other
-                    // chunks pay per-element compares.
-                    const int hi = delta0 + t;
-                    const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
-                    const int t0 = t & ~31;
-                    const int hi_min = delta0 + t0;
-                    const int lo_max = p.window > 0 ? hi_min + 31 - p.window + 1 : INT_MIN;
+                    if (__any_sync(0xffffffffu, m_used == -INFINITY)) {
+                        // No reference yet (the first item's first tiles): the tile's max first.
+                        float mc[8];
 #pragma unroll
-                    for (int cc = 0; cc < kBN; cc += 32) {
-                        if (!(hi_min >= cc + 31 && lo_max <= cc)) {               // not all visible
+                        for (int e = 0; e < 8; ++e) mc[e] = fmaxf(s[2 * e], s[2 * e + 1]);
 #pragma unroll
-                            for (int c = cc; c < cc + 32; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
+                        for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) mc[e] = fmax3f(mc[e], s[c + 2 * e], s[c + 2 * e + 1]);
+                        const float mx = fmaxf(fmax3f(mc[0], mc[1], mc[2]), fmax3f(fmax3f(mc[3], mc[4], mc[5]), mc[6], mc[7]));
+                        if (m_used == -INFINITY) m_used = mx * c1;
+                    }
+                    const float mb = (m_used == -INFINITY) ? 0.0f : m_used;
+                    const uint64_t nm2 = f2_pack(-mb, -mb);
+                    float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[e] = 0;
+#pragma unroll
+                    for (int c = 0; c < kBN; c += 2) {
+                        mc[(c >> 1) & 3] = fmax3f(mc[(c >> 1) & 3], s[c], s[c + 1]);
+                        const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c1x2, nm2);
+                        float p0, p1;
+                        if (((c >> 1) & 7) < kEmuPer8) {
+                            f2_unpack(exp2_fma2(x2), p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(x2, x0, x1);
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
                         }
+                        acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
+                        pk[c / 2] = pack_bf16x2(p0, p1);
                     }
-                }
-                float mc[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mc[e] = fmaxf(s[2 * e], s[2 * e + 1]);
-#pragma unroll
-                for (int c = 16; c < kBN; c += 16)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) mc[e] = fmax3f(mc[e], s[c + 2 * e], s[c + 2 * e + 1]);
-                const float mx = fmaxf(fmax3f(mc[0], mc[1], mc[2]), fmax3f(fmax3f(mc[3], mc[4], mc[5]), mc[6], mc[7]));
-                const float m_tile = mx * c1;
-                const bool grow = m_tile > m_used + kRescaleThreshold;
-                float alpha = 1.0f;
-                if (grow) {
-                    alpha = ex2_approx(m_used - m_tile);
-                    l2 = f2_mul(l2, f2_pack(alpha, alpha));
-                    m_used = m_tile;
-                }
-                if (tt > 0 && __any_sync(0xffffffffu, grow)) {
-                    // O holds every PV up to the previous tile: rescale it in place.
-                    uint32_t ob[32];
-#pragma unroll
-                    for (int c = 0; c < D; c += 32) {
-                        tmem_ld32(o_tm + c, ob);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
-                        tmem_st32(o_tm + c, ob);
+                    const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * c1;
+                    m_seen = fmaxf(m_seen, m_tile);
+                    const bool grow = m_tile > m_used + kRescaleThreshold;
+                    const bool sink = m_tile > -INFINITY && m_seen < m_used - kRefSlack;
+                    if (pass > 0 || !__any_sync(0xffffffffu, grow || sink)) break;
+                    // Re-reference at the running max.  A growing max scales what the row has
+                    // summed so far by 2^(m_used - m_seen); a sinking one is only possible on
+                    // the first tile with a finite max, so what precedes it is masked keys
+                    // and is dropped.
+                    float alpha = 1.0f;
+                    if (grow || sink) {
+                        alpha = grow ? ex2_approx(m_used - m_seen) : 0.0f;
+                        l2 = f2_mul(l2, f2_pack(alpha, alpha));
+                        m_used = m_seen;
                     }
-                    tmem_st_wait();
-                }
-                const float mb = (m_used == -INFINITY) ? 0.0f : m_used;
-                const uint64_t nm2 = f2_pack(-mb, -mb);
-                uint32_t pk[kBN / 2];
-                uint64_t acc[4] = {0, 0, 0, 0};
+                    if (tt > 0) {
+                        // O holds every PV up to the previous tile: rescale it in place.
+                        uint32_t ob[32];
 #pragma unroll
-                for (int c = 0; c < kBN; c += 2) {
-                    const uint64_t x2 = f2_fma(f2_pack(s[c], s[c + 1]), c1x2, nm2);
-                    float p0, p1;
-                    if (((c >> 1) & 7) < kEmuPer8) {
-                        f2_unpack(exp2_fma2(x2), p0, p1);
-                    } else {
-                        float x0, x1;
-                        f2_unpack(x2, x0, x1);
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
+                        for (int c = 0; c < D; c += 32) {
+                            tmem_ld32(o_tm + c, ob);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
+                            tmem_st32(o_tm + c, ob);
+                        }
+                        tmem_st_wait();
                     }
-                    acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
-                    pk[c / 2] = pack_bf16x2(p0, p1);
                 }
                 l2 = f2_add(l2, f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
                 tmem_st32(s_tm, pk);
@@ -746,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(l2, la, lb);
             const float l = la + lb;
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+            m_hint = m_used;
             __nv_bfloat16* orow = p.o + ((static_cast<size_t>(it.b) * p.T + i) * p.Hq + h) * D;
 #pragma unroll
             for (int c = 0; c < D; c += 32) {
@@ -802,42 +863,62 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
 // and zeros elsewhere in the row, with row = (b * T + i) * Hq + h, hp = 0 or h, and
 // pad = 7 - (position & 7): a prefill thread's run of 128 distances for one key tile
 // then starts on a 32-byte boundary.  A block covers 16 rows of one (sequence, head)
-// and 256 distances; each thread one distance for all 16 rows, so a function value is
-// read once and used 16 times.
+// and 1024 distances; each thread holds the C function values of 4 consecutive
+// distances in registers and, row by row, reads the row's C coefficients (four
+// 128-bit shared-memory loads) for 4 C multiply-adds per value.
 constexpr int kCurveRows = 16;
-constexpr int kCurveCols = 256;
+constexpr int kCurveThreads = 256;
+constexpr int kCurveDists = 4;                                  // per thread
+constexpr int kCurveCols = kCurveThreads * kCurveDists;         // per block
 
-__global__ void __launch_bounds__(kCurveCols) bank_rows_kernel(const float* __restrict__ rs,
-                                                               const float* __restrict__ proj,
-                                                               float* __restrict__ out, int B, int T, int Hq,
-                                                               int q_off, int C, int proj_heads, int R, int S) {
-    __shared__ float coef[kCurveRows][kMaxBankC];
+__global__ void __launch_bounds__(kCurveThreads) bank_rows_kernel(const float* __restrict__ rs,
+                                                                  const float* __restrict__ proj,
+                                                                  float* __restrict__ out, int B, int T, int Hq,
+                                                                  int q_off, int C, int proj_heads, int R, int S) {
+    __shared__ __align__(16) float coef[kCurveRows][kMaxBankC];
     const int iblocks = (T + kCurveRows - 1) / kCurveRows;
     const int rb = blockIdx.x;                        // (b, h, row block)
     const int ib = rb % iblocks;
     const int bh = rb / iblocks;
     const int h = bh % Hq, b = bh / Hq;
     const int i_base = ib * kCurveRows;
-    for (int x = threadIdx.x; x < kCurveRows * C; x += blockDim.x) {
-        const int k = x / C, c = x % C;
+    for (int x = threadIdx.x; x < kCurveRows * kMaxBankC; x += blockDim.x) {
+        const int k = x / kMaxBankC, c = x % kMaxBankC;
         const int i = i_base + k;
-        coef[k][c] = i < T ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
+        coef[k][c] = (i < T && c < C) ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
     }
     __syncthreads();
-    const int dist = static_cast<int>(blockIdx.y) * kCurveCols + static_cast<int>(threadIdx.x) - 8;
-    const bool inside = dist >= 0 && dist < R;
-    float pc[kMaxBankC];
+    // Distances dist0 .. dist0+3 (the row's padding reaches 7 below 0 and R+13 above).
+    const int dist0 = static_cast<int>(blockIdx.y) * kCurveCols + static_cast<int>(threadIdx.x) * kCurveDists - 8;
     const float* bank = proj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
+    float pc[kCurveDists][kMaxBankC];
 #pragma unroll
-    for (int c = 0; c < kMaxBankC; ++c) pc[c] = (c < C && inside) ? __ldg(bank + static_cast<size_t>(c) * R + dist) : 0.0f;
+    for (int j = 0; j < kCurveDists; ++j) {
+        const int dist = dist0 + j;
+        const bool inside = dist >= 0 && dist < R;
+#pragma unroll
+        for (int c = 0; c < kMaxBankC; ++c)
+            pc[j][c] = (c < C && inside) ? __ldg(bank + static_cast<size_t>(c) * R + dist) : 0.0f;
+    }
     for (int k = 0; k < kCurveRows; ++k) {
         const int i = i_base + k;
         if (i >= T) break;
-        float acc = 0.0f;
+        float cf[kMaxBankC];
 #pragma unroll
-        for (int c = 0; c < kMaxBankC; ++c) acc = fmaf(coef[k][c], pc[c], acc);   // pc[c] = 0 for c >= C
-        const int x = dist + (7 - ((q_off + i) & 7));
-        if (x >= 0 && x < S) out[((static_cast<size_t>(b) * T + i) * Hq + h) * S + x] = inside ? acc : 0.0f;
+        for (int c = 0; c < kMaxBankC; c += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(&coef[k][c]);
+            cf[c] = v.x, cf[c + 1] = v.y, cf[c + 2] = v.z, cf[c + 3] = v.w;
+        }
+        const int pad = 7 - ((q_off + i) & 7);
+        float* row = out + ((static_cast<size_t>(b) * T + i) * Hq + h) * S;
+#pragma unroll
+        for (int j = 0; j < kCurveDists; ++j) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < kMaxBankC; ++c) acc = fmaf(cf[c], pc[j][c], acc);   // pc = 0 outside [0, R), c >= C
+            const int x = dist0 + j + pad;
+            if (x >= 0 && x < S) row[x] = acc;
+        }
     }
 }
 
@@ -847,13 +928,10 @@ int prefill_bf16_table_copies(int d, int R) {
     return 0;
 }
 
-int prefill_bf16_smem_bytes(int d, int R) {
-    const int nc = prefill_bf16_table_copies(d, R);
-    if (nc == 0) return -1;
-    const int need = smem_bytes_for(d, R, nc);
+int prefill_bf16_smem_bytes(int d, int R, int nc) {
     // Each CTA allocates all 512 TMEM columns: never let two CTAs share an SM
     // (228 KB of shared memory per SM, so more than 114 KB each).
-    return need > 120 * 1024 ? need : 120 * 1024;
+    return std::max(smem_bytes_for(d, R, nc), 120 * 1024);
 }
 
 int prefill_bank_curve_stride(int R) { return ((R + 14) + 7) / 8 * 8; }
@@ -865,7 +943,7 @@ cudaError_t launch_bank_rows(const float* rs, const float* proj, float* curves, 
     const long long rblocks = static_cast<long long>(B) * Hq * ((T + kCurveRows - 1) / kCurveRows);
     if (rblocks > INT32_MAX) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(rblocks), (S + 8 + kCurveCols - 1) / kCurveCols);
-    bank_rows_kernel<<<grid, kCurveCols, 0, stream>>>(rs, proj, curves, B, T, Hq, q_off, C, proj_heads, R, S);
+    bank_rows_kernel<<<grid, kCurveThreads, 0, stream>>>(rs, proj, curves, B, T, Hq, q_off, C, proj_heads, R, S);
     return cudaGetLastError();
 }
 
@@ -873,13 +951,13 @@ cudaError_t launch_prefill_bf16_sm100(const CUtensorMap& tq, const CUtensorMap& 
                                       const PrefillParams& p, int d, int grid, cudaStream_t stream) {
     if (p.curves != nullptr) {
         // The bank form: no staged table (shared memory as for R = 0).
-        const int smem = std::max(smem_bytes_for(d, 0, 0), 120 * 1024);
+        const int smem = prefill_bf16_smem_bytes(d, 0, 0);
         if (d == 128) return launch_variant<128, 0>(tq, tk, tv, p, smem, grid, stream);
         return launch_variant<64, 0>(tq, tk, tv, p, smem, grid, stream);
     }
     const int nc = prefill_bf16_table_copies(d, p.R);
-    const int smem = prefill_bf16_smem_bytes(d, p.R);
-    if (nc == 0 || smem < 0) return cudaErrorInvalidValue;
+    if (nc == 0) return cudaErrorInvalidValue;
+    const int smem = prefill_bf16_smem_bytes(d, p.R, nc);
     if (p.paged) {
         if (d == 128) {
             if (nc == 4) return launch_variant<128, 4, true>(tq, tk, tv, p, smem, grid, stream);
