@@ -862,63 +862,70 @@ cudaError_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const C
 //   out[row * S + pad + dist] = sum_c rs[row, c] * proj[hp, c, dist]   for dist in [0, R)
 // and zeros elsewhere in the row, with row = (b * T + i) * Hq + h, hp = 0 or h, and
 // pad = 7 - (position & 7): a prefill thread's run of 128 distances for one key tile
-// then starts on a 32-byte boundary.  A block covers 16 rows of one (sequence, head)
-// and 1024 distances; each thread holds the C function values of 4 consecutive
-// distances in registers and, row by row, reads the row's C coefficients (four
-// 128-bit shared-memory loads) for 4 C multiply-adds per value.
-constexpr int kCurveRows = 16;
-constexpr int kCurveThreads = 256;
-constexpr int kCurveDists = 4;                                  // per thread
-constexpr int kCurveCols = kCurveThreads * kCurveDists;         // per block
+// then starts on a 32-byte boundary.
+// A block covers the 32 rows of one (sequence, head) in a 256-row span whose positions
+// agree mod 8 (so they share the pad), and its threads the padded positions x (two
+// each, 128 apart): a thread loads the C function values at distance x - pad once and
+// applies them to every row (C multiply-adds per value), and a warp writes 32
+// consecutive floats of a row (whole 128-byte lines).
+constexpr int kCurveRows = 32;   // rows per block, 8 apart (a 256-row span)
+constexpr int kCurveThreads = 128;   // threads per block, 2 positions each (grid y: position blocks)
 
-__global__ void __launch_bounds__(kCurveThreads) bank_rows_kernel(const float* __restrict__ rs,
-                                                                  const float* __restrict__ proj,
-                                                                  float* __restrict__ out, int B, int T, int Hq,
-                                                                  int q_off, int C, int proj_heads, int R, int S) {
+__global__ void __launch_bounds__(kCurveThreads, 8) bank_rows_kernel(const float* __restrict__ rs,
+                                                                     const float* __restrict__ proj,
+                                                                     float* __restrict__ out, int B, int T, int Hq,
+                                                                     int q_off, int C, int proj_heads, int R, int S) {
     __shared__ __align__(16) float coef[kCurveRows][kMaxBankC];
-    const int iblocks = (T + kCurveRows - 1) / kCurveRows;
-    const int rb = blockIdx.x;                        // (b, h, row block)
-    const int ib = rb % iblocks;
-    const int bh = rb / iblocks;
-    const int h = bh % Hq, b = bh / Hq;
-    const int i_base = ib * kCurveRows;
-    for (int x = threadIdx.x; x < kCurveRows * kMaxBankC; x += blockDim.x) {
-        const int k = x / kMaxBankC, c = x % kMaxBankC;
-        const int i = i_base + k;
-        coef[k][c] = (i < T && c < C) ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
+    const int spans = (T + 8 * kCurveRows - 1) / (8 * kCurveRows);
+    int blk = static_cast<int>(blockIdx.x);          // (b, h, span, residue)
+    const int rho = blk & 7;
+    blk >>= 3;
+    const int span = blk % spans;
+    blk /= spans;
+    const int h = blk % Hq, b = blk / Hq;
+    const int i0 = span * 8 * kCurveRows + rho;      // rows i0 + 8m, m < kCurveRows
+    for (int x = threadIdx.x; x < kCurveRows * kMaxBankC; x += kCurveThreads) {
+        const int m = x / kMaxBankC, c = x % kMaxBankC;
+        const int i = i0 + 8 * m;
+        coef[m][c] = (i < T && c < C) ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
     }
     __syncthreads();
-    // Distances dist0 .. dist0+3 (the row's padding reaches 7 below 0 and R+13 above).
-    const int dist0 = static_cast<int>(blockIdx.y) * kCurveCols + static_cast<int>(threadIdx.x) * kCurveDists - 8;
+    // Positions x0 and x0 + 128 of this thread (the second may lie past S).
+    const int x0 = static_cast<int>(blockIdx.y) * 2 * kCurveThreads + static_cast<int>(threadIdx.x);
+    if (i0 >= T || x0 >= S) return;
+    const bool two = x0 + kCurveThreads < S;
+    const int nrows = min(kCurveRows, (T - i0 + 7) / 8);
+    const int pad = 7 - ((q_off + i0) & 7);
     const float* bank = proj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
-    float pc[kCurveDists][kMaxBankC];
+    const size_t row_step = static_cast<size_t>(8) * Hq * S;      // floats between rows i and i + 8
+    float* dst = out + ((static_cast<size_t>(b) * T + i0) * Hq + h) * S + x0;
+    float pc[2][kMaxBankC];
 #pragma unroll
-    for (int j = 0; j < kCurveDists; ++j) {
-        const int dist = dist0 + j;
-        const bool inside = dist >= 0 && dist < R;
+    for (int q = 0; q < 2; ++q) {
+        const int dist = x0 + q * kCurveThreads - pad;
+        const bool inside = dist >= 0 && dist < R && (q == 0 || two);
 #pragma unroll
         for (int c = 0; c < kMaxBankC; ++c)
-            pc[j][c] = (c < C && inside) ? __ldg(bank + static_cast<size_t>(c) * R + dist) : 0.0f;
+            pc[q][c] = (c < C && inside) ? __ldg(bank + static_cast<size_t>(c) * R + dist) : 0.0f;
     }
-    for (int k = 0; k < kCurveRows; ++k) {
-        const int i = i_base + k;
-        if (i >= T) break;
-        float cf[kMaxBankC];
+    // Row by row: the row's C coefficients (broadcast shared-memory loads) serve both
+    // positions; each sum is split in halves (4 independent chains per row).
+    for (int m = 0; m < nrows; ++m, dst += row_step) {
+        float lo[2] = {0.0f, 0.0f}, hi[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int c = 0; c < kMaxBankC; c += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(&coef[k][c]);
-            cf[c] = v.x, cf[c + 1] = v.y, cf[c + 2] = v.z, cf[c + 3] = v.w;
+        for (int c = 0; c < kMaxBankC / 2; c += 4) {
+            const float4 u = *reinterpret_cast<const float4*>(&coef[m][c]);
+            const float4 w = *reinterpret_cast<const float4*>(&coef[m][c + kMaxBankC / 2]);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                lo[q] = fmaf(u.x, pc[q][c], lo[q]), lo[q] = fmaf(u.y, pc[q][c + 1], lo[q]);
+                lo[q] = fmaf(u.z, pc[q][c + 2], lo[q]), lo[q] = fmaf(u.w, pc[q][c + 3], lo[q]);
+                hi[q] = fmaf(w.x, pc[q][c + 8], hi[q]), hi[q] = fmaf(w.y, pc[q][c + 9], hi[q]);
+                hi[q] = fmaf(w.z, pc[q][c + 10], hi[q]), hi[q] = fmaf(w.w, pc[q][c + 11], hi[q]);
+            }
         }
-        const int pad = 7 - ((q_off + i) & 7);
-        float* row = out + ((static_cast<size_t>(b) * T + i) * Hq + h) * S;
-#pragma unroll
-        for (int j = 0; j < kCurveDists; ++j) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int c = 0; c < kMaxBankC; ++c) acc = fmaf(cf[c], pc[j][c], acc);   // pc = 0 outside [0, R), c >= C
-            const int x = dist0 + j + pad;
-            if (x >= 0 && x < S) row[x] = acc;
-        }
+        dst[0] = lo[0] + hi[0];
+        if (two) dst[kCurveThreads] = lo[1] + hi[1];
     }
 }
 
@@ -940,9 +947,9 @@ cudaError_t launch_bank_rows(const float* rs, const float* proj, float* curves, 
                              int proj_heads, int R, cudaStream_t stream) {
     if (B < 1 || T < 1 || R < 1) return cudaSuccess;
     const int S = prefill_bank_curve_stride(R);
-    const long long rblocks = static_cast<long long>(B) * Hq * ((T + kCurveRows - 1) / kCurveRows);
-    if (rblocks > INT32_MAX) return cudaErrorInvalidValue;
-    dim3 grid(static_cast<unsigned>(rblocks), (S + 8 + kCurveCols - 1) / kCurveCols);
+    const long long blocks = static_cast<long long>(B) * Hq * ((T + 8 * kCurveRows - 1) / (8 * kCurveRows)) * 8;
+    if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(blocks), (S + 2 * kCurveThreads - 1) / (2 * kCurveThreads));
     bank_rows_kernel<<<grid, kCurveThreads, 0, stream>>>(rs, proj, curves, B, T, Hq, q_off, C, proj_heads, R, S);
     return cudaGetLastError();
 }

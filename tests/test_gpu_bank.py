@@ -78,6 +78,7 @@ BF16_CASES = [
     (1, 513, 6, 3, 64, 0, 300, 5, 1, 100),      # odd group, d = 64, temperature, R not a tile multiple
     (1, 1, 4, 4, 128, 0, 16, 3, 1, 0),          # a single token
     (1, 260, 4, 2, 128, 0, 1000, 16, 1, 0),     # R beyond the sequence
+    (1, 150, 4, 2, 128, 0, 77, 7, 4, 0),        # R odd (the curve kernel's scalar loads)
 ]
 
 
@@ -120,6 +121,21 @@ def test_bf16_bank_of_one_function_per_head_matches_rank1():
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
     assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_bf16_bank_unaligned_proj_matches_aligned():
+    """proj at a 4-byte offset (not 16-byte aligned) takes the curve kernel's scalar
+    loads and gives the same output, bit for bit."""
+    B, T, Hq, Hkv, d, R, C = 1, 300, 4, 2, 128, 256, 16
+    q, k, v, rs, proj = _bank_inputs(B, T, Hq, Hkv, d, R, C, 1, seed=17)
+    buf = torch.empty(proj.numel() + 1, dtype=torch.float32, device="cuda")
+    shifted = buf[1:].view(proj.shape)
+    shifted.copy_(proj)
+    assert shifted.data_ptr() % 16 != 0 and shifted.is_contiguous()
+    o1 = ops.attn_fwd_bank(q, k, v, rs, proj, 0, R, 0.1)
+    o2 = ops.attn_fwd_bank(q, k, v, rs, shifted, 0, R, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
 
 
 def test_bf16_bank_workspace_is_not_read_before_written():

@@ -183,3 +183,23 @@ def test_backward_writes_stay_inside(dtype, T, window):
     for n, gb in g.items():
         gb.check(n)
     ws.check("workspace", fully_written=False)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,d,window,R,C,proj_heads", [
+    (1, 1, 4, 2, 128, 0, 16, 3, 1),          # a single token
+    (2, 129, 6, 2, 128, 0, 99, 16, 6),       # one tile plus one row, R not a multiple of 4
+    (1, 300, 8, 1, 64, 128, 128, 5, 1),      # windowed, d = 64
+])
+def test_bank_prefill_writes_stay_inside(B, T, Hq, Hkv, d, window, R, C, proj_heads):
+    x = _x(B, T, Hq, Hkv, d, R, seed=T + C)
+    rs = synth.normal((B, T, Hq, C), T, "rs", std=0.25, device="cuda")
+    proj = synth.normal((proj_heads, C, R), T, "proj", std=0.5, device="cuda")
+    need = ops.fwd_bank_workspace_size(B, T, Hq, R, ops.RELBIAS_BF16)
+    ws = Guarded((need,), torch.uint8)
+    o = Guarded((B, T, Hq, d), torch.bfloat16)
+    lse = Guarded((B, Hq, T), torch.float32)
+    ops.attn_fwd_bank(x["q"], x["k"], x["v"], rs, proj, window, R, 1.0 / math.sqrt(d), out=o.t, lse=lse.t,
+                      workspace=ws.t)
+    o.check("o")
+    lse.check("lse")
+    ws.check("workspace", fully_written=False)
