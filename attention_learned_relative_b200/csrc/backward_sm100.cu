@@ -433,7 +433,8 @@ __global__ void __launch_bounds__(kBqThreads, 1)
 
 // ------------------------------------------------------------------------- dK/dV kernel
 
-constexpr int kBkThreads = 192;   // warps 0-3 key rows, 4 TMA producer, 5 MMA issuer
+constexpr int kBkThreads = 320;   // warps 0-7 key rows (two per TMEM lane quadrant), 8 TMA producer, 9 MMA issuer
+constexpr int kBkRowWarps = 8;
 
 template <int D>
 struct BkLayout {
@@ -443,7 +444,8 @@ struct BkLayout {
     static constexpr int kQ = kV + kTile;              // 2 stages
     static constexpr int kDO = kQ + 2 * kTile;         // 2 stages
     static constexpr int kCol = kDO + 2 * kTile;       // per-column constants, 2 buffers of [128] float8
-    static constexpr int kDw = kCol + 2 * kBM * 32;    // table gradient accumulator [R]
+    static constexpr int kEm = kCol + 2 * kBM * 32;    // per key-row warp: its diagonal sums by column [8][128]
+    static constexpr int kDw = kEm + kBkRowWarps * kBN * 4;   // table gradient accumulator [R]
 };
 
 struct BkBars {
@@ -509,6 +511,21 @@ __device__ __forceinline__ BkItem bk_item_at(const PrefillParams& p, int k) {
     return it;
 }
 
+// dV += P^T dO (or dK += dS^T Q) with P^T from tensor memory, where the two column
+// halves of the step wrote their packed bf16 values at columns [0, 32) and [64, 96):
+// each half packs over its own fp32 columns only, so neither overwrites logits the
+// other has yet to read.
+template <int D>
+__device__ __forceinline__ void issue_acc_split(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t b_addr,
+                                                uint32_t idesc, bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < kBM / 16; ++kk) {
+        const uint64_t b = smem_desc_sw128(b_addr + kk * 16 * 128, Layout<D>::kBox, 1024);
+        const uint32_t a = p_tmem + kk * 8 + (kk >= kBM / 32 ? 32 : 0);
+        if (leader) umma_ts(d_tmem, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
 // Query row qt * 128 + t of head (g * G + hl): its (r, LSE, D) (zeros past T).
 __device__ __forceinline__ float3 bk_col_inputs(const PrefillParams& p, const BwdTcParams& bp, const BkItem& it, int hl,
                                                 int qt, int t) {
@@ -531,6 +548,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
     const int tstride = tab_stride(p.R, NCOPY);
     const int tslot = NCOPY * tstride;
     float* dw_s = reinterpret_cast<float*>(smem + L::kDw);
+    float* emit = reinterpret_cast<float*>(smem + L::kEm);
     const int dw_len = ((p.R + 3) / 4) * 4;
     float* wtab = dw_s + dw_len;
     BkBars* bars = reinterpret_cast<BkBars*>(reinterpret_cast<uint8_t*>(wtab) + tslot * 4);
@@ -548,20 +566,20 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             mbar_init(&bars->do_empty[s], 1);
         }
         mbar_init(&bars->sdp_full, 1);
-        mbar_init(&bars->pd_ready, kBM / 32);
+        mbar_init(&bars->pd_ready, kBkRowWarps);
         mbar_init(&bars->acc_final, 1);
-        mbar_init(&bars->acc_free, kBM / 32);
-        mbar_init(&bars->col_sync, kBM / 32);
+        mbar_init(&bars->acc_free, kBkRowWarps);
+        mbar_init(&bars->col_sync, kBkRowWarps);
         mbar_init(&bars->mma_done, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
         tc_fence_before();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_k);
@@ -571,11 +589,12 @@ __global__ void __launch_bounds__(kBkThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_base;
     const int nitems = bk_items_of_cta(p);
-    // Tensor memory: S^T [0, 128) (P^T over it), dP^T [128, 256) (dS^T over it),
+    // Tensor memory: S^T [0, 128) (P^T over it, packed bf16: queries 0-63 at [0, 32),
+    // 64-127 at [64, 96)), dP^T [128, 256) (dS^T over it, likewise),
     // dV [256, 256 + D), dK [384, 384 + D).  Steps s run over (head of the group, query
     // tile) within an item, and across items.
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         const bool leader = elect_one();
         bool ok = true;
@@ -619,7 +638,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             mbar_drain_wait(&bars->q_full[n & 1], (n >> 1) & 1);
             mbar_drain_wait(&bars->do_full[n & 1], (n >> 1) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         const bool leader = elect_one();
         const uint32_t idesc_s = idesc_bf16_f32(kBM, kBM, false, false);
@@ -651,8 +670,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (!(ok = warp_all(mbar_wait(&bars->pd_ready, ns & 1, abort_flag)))) break;
                 tc_fence_after();
                 // dV += P^T dO and dK += dS^T Q: query rows on the K dimension.
-                issue_pv<D>(leader, dv_tm, st_tm, do_addr, idesc_acc, s > 0);
-                issue_pv<D>(leader, dk_tm, dpt_tm, q_addr, idesc_acc, s > 0);
+                issue_acc_split<D>(leader, dv_tm, st_tm, do_addr, idesc_acc, s > 0);
+                issue_acc_split<D>(leader, dk_tm, dpt_tm, q_addr, idesc_acc, s > 0);
                 if (leader) {
                     umma_commit(&bars->q_empty[st]);
                     umma_commit(&bars->do_empty[st]);
@@ -668,7 +687,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         mbar_drain_wait(&bars->mma_done, 0);
     } else {
         // ---------------------------------------------------------------- key rows
-        const int t = threadIdx.x;   // key k0 + t of the tile (TMEM lane)
+        const int t = threadIdx.x & (kBM - 1);   // key k0 + t of the tile (TMEM lane)
+        const int half = threadIdx.x >> 7;        // columns [64 half, 64 half + 64) of each step
         const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
         const uint32_t st_tm = tmem_base + lane_off, dpt_tm = tmem_base + lane_off + 128,
                        dv_tm = tmem_base + lane_off + 256, dk_tm = tmem_base + lane_off + 384;
@@ -699,12 +719,12 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
                 if (p.R > 0) {
                     const float* wrow = p.w + static_cast<size_t>(h) * p.R;
-                    for (int x = t; x < tslot; x += kBM) {
+                    for (int x = threadIdx.x; x < tslot; x += kBkRowWarps * 32) {
                         const int cp = x / tstride;
                         const int dd = x - cp * tstride + cp + kBkDmin;
                         wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(wrow + dd) : 0.0f;
                     }
-                    for (int x = t; x < dw_len; x += kBM) dw_s[x] = 0.0f;
+                    for (int x = threadIdx.x; x < dw_len; x += kBkRowWarps * 32) dw_s[x] = 0.0f;
                 }
                 for (int qt = qt_lo; qt <= qt_hi; ++qt, ++ns) {
                     const int i0 = qt * kBM;
@@ -735,8 +755,9 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                         }
                         const float c1 = p.scale_log2 * tau;
                         const float ri = cur.x;
-                        cb[2 * t] = make_float4(c1, ri * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z);
-                        cb[2 * t + 1] = make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
+                        // (the two halves write one float4 each)
+                        cb[2 * t + half] = half == 0 ? make_float4(c1, ri * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z)
+                                                     : make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
                     }
                     if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
                     if (!(ok = warp_all(mbar_wait(&bars->sdp_full, ns & 1, abort_flag)))) break;
@@ -747,8 +768,16 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     const int cp = y0 & (NCOPY - 1);
                     const float* run = wtab + cp * tstride + (y0 - cp);
                     const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBN - 1 >= p.window);
+                    // dw: the cells of a distance lie on a diagonal (key t, column c) -> (t+1, c+1).
+                    // A conveyor sums them: per column, zdw = g + (lane above's zdw), so lane 31
+                    // holds a finished sum of its warp's part of one diagonal each column
+                    // (stashed by column in `em`), and after the half's last column lanes 0-30
+                    // hold the diagonals that leave there.  Each warp then adds 2 + 1
+                    // distinct-address rows of sums to dw instead of one per cell.
+                    float zdw = 0.0f;
+                    float* em = emit + (threadIdx.x >> 5) * kBN;
 #pragma unroll 1
-                    for (int ch = 0; ch < kBM / 32; ++ch) {
+                    for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
                         uint32_t sv[32], dv[32];
                         tmem_ld32(st_tm + 32 * ch, sv);
                         tmem_ld32(dpt_tm + 32 * ch, dv);
@@ -770,23 +799,41 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                                 const float dl = pv * (__uint_as_float(dv[e + k]) - a.w);
                                 pr[k] = pv;
                                 dsv[k] = dl * b2.x;
-                                if (biased && dist >= 0 && dist < p.R && dl != 0.0f) atomicAdd(dw_s + dist, dl * b2.y);
+                                if (biased) {
+                                    const float g = (dist >= 0 && dist < p.R) ? dl * b2.y : 0.0f;
+                                    const float up = __shfl_up_sync(0xffffffffu, zdw, 1);
+                                    zdw = g + (lane > 0 ? up : 0.0f);
+                                    if (lane == 31) em[c] = zdw;
+                                }
                             }
                             pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
                             pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
                         }
-                        tmem_st16(st_tm + 16 * ch, pp);
-                        tmem_st16(dpt_tm + 16 * ch, pd);
+                        tmem_st16(st_tm + 16 * ch + 32 * half, pp);
+                        tmem_st16(dpt_tm + 16 * ch + 32 * half, pd);
                     }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->pd_ready);
+                    if (biased) {
+                        // Lane 31's sums: distance delta0 + c - (32 w + 31) at column c.
+                        const int dbase = delta0 - ((t & ~31) + 31);
+#pragma unroll
+                        for (int q = 2 * half; q < 2 * half + 2; ++q) {
+                            const int d = dbase + lane + 32 * q;
+                            if (d >= 0 && d < p.R) atomicAdd(dw_s + d, em[lane + 32 * q]);
+                        }
+                        // Diagonals leaving at the half's last column: distance delta0 + 64 half + 63 - t.
+                        const int d = delta0 + 64 * half + 63 - t;
+                        if (lane < 31 && d >= 0 && d < p.R) atomicAdd(dw_s + d, zdw);
+                        __syncwarp();
+                    }
                 }
                 if (!ok) break;
                 // This head's table gradient from this key tile, into the output.
                 if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
-                for (int x = t; x < p.R; x += kBM)
+                for (int x = threadIdx.x; x < p.R; x += kBkRowWarps * 32)
                     if (dw_s[x] != 0.0f) atomicAdd(bp.dw + static_cast<size_t>(h) * p.R + x, dw_s[x]);
             }
             if (!ok) break;
@@ -795,7 +842,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             tc_fence_after();
             const size_t krow = (static_cast<size_t>(it.b) * p.T + (key_ok ? j : 0)) * p.Hkv + it.g;
 #pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
+            for (int c = half * D / 2; c < (half + 1) * D / 2; c += 32) {
                 uint32_t a[32], b[32];
                 tmem_ld32(dk_tm + c, a);
                 tmem_ld32(dv_tm + c, b);
@@ -819,7 +866,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
     }
 
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
     }
