@@ -33,7 +33,8 @@ namespace {
 
 // ------------------------------------------------------------------------- dQ kernel
 
-constexpr int kBqThreads = 192;   // warps 0-3 rows, 4 TMA producer, 5 MMA issuer
+constexpr int kBqThreads = 320;   // warps 0-7 rows (two per TMEM lane quadrant), 8 TMA producer, 9 MMA issuer
+constexpr int kBqRowWarps = 8;
 
 template <int D>
 struct BqLayout {
@@ -84,11 +85,12 @@ struct TileCursor {
     __device__ __forceinline__ int j0() const { return j_first + t * kBN; }
 };
 
-// D_i = dO_i . O_i for every row (b, i, h), into dvec [B, Hq, T]: one warp per row.
+// D_i = dO_i . O_i for every row (b, i, h), into dvec [B, Hq, T], and dr zeroed: one
+// warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout, float* __restrict__ dvec,
-                                                       int B, int T, int Hq) {
+                                                       float* __restrict__ dr, int B, int T, int Hq) {
     const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // (b * T + i) * Hq + h
     const int lane = threadIdx.x & 31;
     if (row >= static_cast<long long>(B) * T * Hq) return;
@@ -106,6 +108,7 @@ __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __re
         const long long bi = row / Hq;
         const int i = static_cast<int>(bi % T), b = static_cast<int>(bi / T);
         dvec[(static_cast<size_t>(b) * Hq + h) * T + i] = acc;
+        dr[row] = 0.0f;   // the dQ kernel's two column halves add into it
     }
 }
 
@@ -117,6 +120,21 @@ __device__ __forceinline__ float3 bq_row_inputs(const PrefillParams& p, const Bw
     const size_t hrow = (static_cast<size_t>(it.b) * p.Hq + h) * p.T + i;
     return make_float3(__ldg(bp.dvec + hrow), __ldg(bp.lse + hrow),
                        __ldg(p.r + (static_cast<size_t>(it.b) * p.T + i) * p.Hq + h));
+}
+
+// An accumulating MMA (dQ += dS K, dV += P^T dO, dK += dS^T Q) whose A operand is bf16
+// in tensor memory, written by two warps per lane quadrant: the warp of column half h
+// packs its 64 values of a row at columns [64 h, 64 h + 32), over fp32 columns only it
+// has read, so neither warp overwrites values the other has yet to load.
+template <int D>
+__device__ __forceinline__ void issue_acc_split(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t b_addr,
+                                                uint32_t idesc, bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < kBM / 16; ++kk) {
+        const uint64_t b = smem_desc_sw128(b_addr + kk * 16 * 128, Layout<D>::kBox, 1024);
+        const uint32_t a = p_tmem + kk * 8 + (kk >= kBM / 32 ? 32 : 0);
+        if (leader) umma_ts(d_tmem, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
 }
 
 template <int D, int NCOPY>
@@ -147,21 +165,21 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             mbar_init(&bars->v_empty[s], 1);
         }
         mbar_init(&bars->sdp_full, 1);
-        mbar_init(&bars->dp_free, kBM / 32);
-        mbar_init(&bars->ds_ready, kBM / 32);
+        mbar_init(&bars->dp_free, kBqRowWarps);
+        mbar_init(&bars->ds_ready, kBqRowWarps);
         mbar_init(&bars->dq_final, 1);
-        mbar_init(&bars->dq_free, kBM / 32);
-        mbar_init(&bars->tab_sync, kBM / 32);
+        mbar_init(&bars->dq_free, kBqRowWarps);
+        mbar_init(&bars->tab_sync, kBqRowWarps);
         mbar_init(&bars->mma_done, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
         tc_fence_before();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_do);
         prefetch_tmap(&tm_k);
@@ -173,7 +191,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
     const int nitems = items_of_cta(p);
     // Tensor memory: S(g) in [128 * (g & 1), +128), dP [256, 384), dQ [384, 384 + D).
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         const bool leader = elect_one();
         bool ok = true;
@@ -233,7 +251,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             mbar_drain_wait(&bars->k_full[n & 1], (n >> 1) & 1);
             mbar_drain_wait(&bars->v_full[n & 1], (n >> 1) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         // Per tile g the issue order is QK(g+1), dP(g+1), dQ(g): the next tile's S and dP
         // are computed while the rows' warps work on tile g (S is double-buffered; dP is
@@ -277,8 +295,8 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             tc_fence_after();
             // dQ += dS K: dS (bf16 pairs over the first 64 columns of S(g)) times the key tile,
             // keys on the K dimension (MN-major operand, as V in the forward's PV).
-            issue_pv<D>(leader, dq_tm, tmem_base + 128 * (g & 1), smem_u32(smem + L::kK + (g & 1) * L::kTile),
-                        idesc_dq, !cur.first());
+            issue_acc_split<D>(leader, dq_tm, tmem_base + 128 * (g & 1),
+                               smem_u32(smem + L::kK + (g & 1) * L::kTile), idesc_dq, !cur.first());
             if (leader) umma_commit(&bars->k_empty[g & 1]);
             if (leader && cur.last()) umma_commit(&bars->dq_final);
             if (!have_next) break;
@@ -288,7 +306,8 @@ __global__ void __launch_bounds__(kBqThreads, 1)
         mbar_drain_wait(&bars->mma_done, 0);
     } else {
         // ---------------------------------------------------------------- rows
-        const int t = threadIdx.x;                       // row t of the query tile (TMEM lane)
+        const int t = threadIdx.x & (kBM - 1);           // row t of the query tile (TMEM lane)
+        const int half = threadIdx.x >> 7;               // key columns [64 half, 64 half + 64) of each tile
         const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
         const uint32_t dp_tm = tmem_base + lane_off + 256, dq_tm = tmem_base + lane_off + 384;
         const int cmax = tab_cmax(p.R);
@@ -310,7 +329,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 staged_head = h;
                 if (!(ok = tab_meet(&bars->tab_sync, tab_phase, abort_flag))) break;
                 const float* wrow = p.w + static_cast<size_t>(h) * p.R;
-                for (int x = t; x < tslot; x += kBM) {
+                for (int x = threadIdx.x; x < tslot; x += kBqRowWarps * 32) {
                     const int cp = x / tstride;
                     const int dd = cmax - (x - cp * tstride + cp);
                     wtab[x] = (dd >= 0 && dd < p.R) ? __ldg(wrow + dd) : 0.0f;
@@ -341,9 +360,9 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 const uint32_t s_tm = tmem_base + lane_off + 128 * (g & 1);
                 if (!(ok = warp_all(mbar_wait(&bars->sdp_full, g & 1, abort_flag)))) break;
                 tc_fence_after();
-                uint32_t dp[kBN];
+                uint32_t dp[kBN / 2];   // this half's columns
 #pragma unroll
-                for (int c = 0; c < kBN; c += 32) tmem_ld32(dp_tm + c, dp + c);
+                for (int c = 0; c < kBN / 2; c += 32) tmem_ld32(dp_tm + 64 * half + c, dp + c);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -356,7 +375,8 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 const int hi = delta0 + t;
                 const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
 #pragma unroll
-                for (int ch = 0; ch < kBN / 32; ++ch) {
+                for (int lc = 0; lc < 2; ++lc) {
+                    const int ch = 2 * half + lc;   // this half's chunks of 32 columns
                     uint32_t sv[32];
                     tmem_ld32(s_tm + 32 * ch, sv);
                     tmem_ld_wait();
@@ -384,13 +404,13 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                             const float x = fmaf(__uint_as_float(sv[e + k]), c1, fmaf(rb, w4[k], -lse2));
                             const bool vis = !edge || (c <= hi && c >= lo);
                             const float pr = vis ? ex2_approx(x) : 0.0f;
-                            dl[k] = pr * (__uint_as_float(dp[c]) - Di);
+                            dl[k] = pr * (__uint_as_float(dp[32 * lc + e + k]) - Di);
                             dr_acc = fmaf(dl[k], w4[k], dr_acc);
                         }
                         pk[e / 2] = pack_bf16x2(dl[0] * ds_scale, dl[1] * ds_scale);
                         pk[e / 2 + 1] = pack_bf16x2(dl[2] * ds_scale, dl[3] * ds_scale);
                     }
-                    tmem_st16(s_tm + 16 * ch, pk);
+                    tmem_st16(s_tm + 16 * ch + 32 * half, pk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -399,13 +419,14 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             }
             if (!ok) break;
 
-            // Epilogue: dr and the row of dq.
-            if (row_ok) bp.dr[row] = dr_acc * tau;
+            // Epilogue: dr (the two halves' partial sums added into the zeros the D kernel
+            // wrote; a sum of two terms does not depend on their order) and the row of dq.
+            if (row_ok) atomicAdd(bp.dr + row, dr_acc * tau);
             if (!(ok = warp_all(mbar_wait(&bars->dq_final, item_it & 1, abort_flag)))) break;
             tc_fence_after();
             float* dqrow = bp.dq + row * D;
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
+            for (int c = half * D / 2; c < (half + 1) * D / 2; c += 32) {
                 uint32_t v[32];
                 tmem_ld32(dq_tm + c, v);
                 tmem_ld_wait();
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
     }
 
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
     }
@@ -509,21 +530,6 @@ __device__ __forceinline__ BkItem bk_item_at(const PrefillParams& p, int k) {
     it.b = rem / p.Hkv;
     it.g = rem - it.b * p.Hkv;
     return it;
-}
-
-// dV += P^T dO (or dK += dS^T Q) with P^T from tensor memory, where the two column
-// halves of the step wrote their packed bf16 values at columns [0, 32) and [64, 96):
-// each half packs over its own fp32 columns only, so neither overwrites logits the
-// other has yet to read.
-template <int D>
-__device__ __forceinline__ void issue_acc_split(bool leader, uint32_t d_tmem, uint32_t p_tmem, uint32_t b_addr,
-                                                uint32_t idesc, bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < kBM / 16; ++kk) {
-        const uint64_t b = smem_desc_sw128(b_addr + kk * 16 * 128, Layout<D>::kBox, 1024);
-        const uint32_t a = p_tmem + kk * 8 + (kk >= kBM / 32 ? 32 : 0);
-        if (leader) umma_ts(d_tmem, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
 }
 
 // Query row qt * 128 + t of head (g * G + hl): its (r, LSE, D) (zeros past T).
@@ -907,8 +913,8 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const C
                           const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
                           const BwdTcParams& bp, int grid, cudaStream_t stream) {
     const long long rows = static_cast<long long>(p_dq.B) * p_dq.T * p_dq.Hq;
-    bwd_dvec_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(bp.o, bp.dout, bp.dvec, p_dq.B,
-                                                                                 p_dq.T, p_dq.Hq);
+    bwd_dvec_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(bp.o, bp.dout, bp.dvec, bp.dr,
+                                                                                 p_dq.B, p_dq.T, p_dq.Hq);
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
     const int nc = bq_copies<D>(p_dq.R);
