@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __re
         const long long bi = row / Hq;
         const int i = static_cast<int>(bi % T), b = static_cast<int>(bi / T);
         dvec[(static_cast<size_t>(b) * Hq + h) * T + i] = acc;
-        dr[row] = 0.0f;   // the dQ kernel's two column halves add into it
+        if (dr != nullptr) dr[row] = 0.0f;   // the dQ kernel's two column halves add into it
     }
 }
 
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             const int h = it.g * p.G + it.hp;
             const float3 cur = nxt;
             if (item_it + 1 < nitems) nxt = bq_row_inputs(p, bp, item_at(p, item_it + 1), t);
-            if (h != staged_head) {
+            if (NCOPY > 0 && h != staged_head) {
                 staged_head = h;
                 if (!(ok = tab_meet(&bars->tab_sync, tab_phase, abort_flag))) break;
                 const float* wrow = p.w + static_cast<size_t>(h) * p.R;
@@ -350,7 +350,13 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 if (n > p.temp_n0) tau = __logf(static_cast<float>(n)) * p.inv_log_n0;
             }
             const float c1 = p.scale_log2 * tau;
-            const float rb = cur.z * p.inv_scale * c1;   // bias, log2 units
+            // Bias coefficient, log2 units: r_i / scale (rank-1 form) or 1 / scale (the
+            // bank form, whose curve holds the whole bias).
+            const float rb = (NCOPY > 0 ? cur.z : 1.0f) * p.inv_scale * c1;
+            // The bank form: the row's curve and its gradient, at distance 0 (padded rows).
+            const size_t crow = row * static_cast<size_t>(bp.curve_stride) + (7 - (i & 7));
+            const float* curve = NCOPY == 0 ? bp.curves + crow : nullptr;
+            float* dcurve = NCOPY == 0 ? bp.dcv + crow : nullptr;
             const float ds_scale = tau * bp.scale;   // dS = tau * scale * dl, the dQ MMA's operand
             float dr_acc = 0.0f;                     // sum_j dl_j w[h, i-j]
 
@@ -363,7 +369,8 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 uint32_t dp[kBN / 2];   // this half's columns
 #pragma unroll
                 for (int c = 0; c < kBN / 2; c += 32) tmem_ld32(dp_tm + 64 * half + c, dp + c);
-                tmem_ld_wait();
+                tmem_ld_wait_regs(dp);
+                tmem_regs_fence(dp + 32);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->dp_free);
@@ -375,16 +382,27 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 const int hi = delta0 + t;
                 const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
 #pragma unroll
+                uint32_t pk2[2][16];   // both chunks' dS: live until the stores are waited for
+#pragma unroll
                 for (int lc = 0; lc < 2; ++lc) {
                     const int ch = 2 * half + lc;   // this half's chunks of 32 columns
+                    uint32_t* pk = pk2[lc];
                     uint32_t sv[32];
                     tmem_ld32(s_tm + 32 * ch, sv);
-                    tmem_ld_wait();
-                    uint32_t pk[16];
+                    tmem_ld_wait_regs(sv);
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
                         float w4[4] = {0.f, 0.f, 0.f, 0.f};
-                        if (biased) {
+                        // Distances of columns c .. c+3 are dlo4+3 .. dlo4 (a 16-byte aligned
+                        // group of the padded curve row).
+                        const int dlo4 = delta0 + t - (32 * ch + e) - 3;
+                        const bool in_curve = row_ok && dlo4 + 3 >= 0 && dlo4 < p.R;
+                        if (NCOPY == 0) {
+                            if (biased && in_curve) {
+                                const float4 v = __ldg(reinterpret_cast<const float4*>(curve + dlo4));
+                                w4[0] = v.w, w4[1] = v.z, w4[2] = v.y, w4[3] = v.x;
+                            }
+                        } else if (biased) {
                             if constexpr (NCOPY == 4) {
                                 const float4 v = *reinterpret_cast<const float4*>(run + 32 * ch + e);
                                 w4[0] = v.x, w4[1] = v.y, w4[2] = v.z, w4[3] = v.w;
@@ -405,15 +423,25 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                             const bool vis = !edge || (c <= hi && c >= lo);
                             const float pr = vis ? ex2_approx(x) : 0.0f;
                             dl[k] = pr * (__uint_as_float(dp[32 * lc + e + k]) - Di);
-                            dr_acc = fmaf(dl[k], w4[k], dr_acc);
+                            if constexpr (NCOPY > 0) dr_acc = fmaf(dl[k], w4[k], dr_acc);
                         }
+                        if (NCOPY == 0 && biased && in_curve)
+                            *reinterpret_cast<float4*>(dcurve + dlo4) =
+                                make_float4(tau * dl[3], tau * dl[2], tau * dl[1], tau * dl[0]);
                         pk[e / 2] = pack_bf16x2(dl[0] * ds_scale, dl[1] * ds_scale);
                         pk[e / 2 + 1] = pack_bf16x2(dl[2] * ds_scale, dl[3] * ds_scale);
                     }
                     tmem_st16(s_tm + 16 * ch + 32 * half, pk);
                 }
                 tmem_st_wait();
+                tmem_regs_keep16(pk2[0]);
+                tmem_regs_keep16(pk2[1]);
                 tc_fence_before();
+                // S is double-buffered and dP(g+1) needs only dp_free(g), so a warp can
+                // reach this arrival for tile g while another has yet to arrive for g-1.
+                // Arrivals for two tiles must not mix in one phase: wait until phase g-1
+                // (every warp's dS(g-1)) is complete before arriving for g.
+                if (g > 0 && !(ok = warp_all(mbar_wait(&bars->ds_ready, (g - 1) & 1, abort_flag)))) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->ds_ready);
             }
@@ -421,7 +449,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
 
             // Epilogue: dr (the two halves' partial sums added into the zeros the D kernel
             // wrote; a sum of two terms does not depend on their order) and the row of dq.
-            if (row_ok) atomicAdd(bp.dr + row, dr_acc * tau);
+            if (NCOPY > 0 && row_ok) atomicAdd(bp.dr + row, dr_acc * tau);
             if (!(ok = warp_all(mbar_wait(&bars->dq_final, item_it & 1, abort_flag)))) break;
             tc_fence_after();
             float* dqrow = bp.dq + row * D;
@@ -429,7 +457,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
             for (int c = half * D / 2; c < (half + 1) * D / 2; c += 32) {
                 uint32_t v[32];
                 tmem_ld32(dq_tm + c, v);
-                tmem_ld_wait();
+                tmem_ld_wait_regs(v);
                 if (row_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
@@ -723,7 +751,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const int h = it.g * p.G + hl;
                 // This head's table (ascending) and a zeroed dw accumulator.
                 if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
-                if (p.R > 0) {
+                if (NCOPY > 0 && p.R > 0) {
                     const float* wrow = p.w + static_cast<size_t>(h) * p.R;
                     for (int x = threadIdx.x; x < tslot; x += kBkRowWarps * 32) {
                         const int cp = x / tstride;
@@ -762,7 +790,9 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                         const float c1 = p.scale_log2 * tau;
                         const float ri = cur.x;
                         // (the two halves write one float4 each)
-                        cb[2 * t + half] = half == 0 ? make_float4(c1, ri * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z)
+                        // (the bank form's curve holds the whole bias: coefficient 1 / scale)
+                        const float rcoef = NCOPY > 0 ? ri : 1.0f;
+                        cb[2 * t + half] = half == 0 ? make_float4(c1, rcoef * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z)
                                                      : make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
                     }
                     if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
@@ -774,6 +804,14 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     const int cp = y0 & (NCOPY - 1);
                     const float* run = wtab + cp * tstride + (y0 - cp);
                     const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBN - 1 >= p.window);
+                    // The bank form: query row i0 + c's curve at distance delta0 + c - t is
+                    // cstep[c * cstride - (c & 7)] (rows (b, i, h) of curve_stride floats, the
+                    // row of position i padded by 7 - (i & 7)).
+                    const size_t cstride = static_cast<size_t>(p.Hq) * bp.curve_stride + 1;
+                    const float* cstep =
+                        NCOPY == 0 ? bp.curves + ((static_cast<size_t>(it.b) * p.T + i0) * p.Hq + h) * bp.curve_stride +
+                                         delta0 + 7 - t
+                                   : nullptr;
                     // dw: the cells of a distance lie on a diagonal (key t, column c) -> (t+1, c+1).
                     // A conveyor sums them: per column, zdw = g + (lane above's zdw), so lane 31
                     // holds a finished sum of its warp's part of one diagonal each column
@@ -787,7 +825,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                         uint32_t sv[32], dv[32];
                         tmem_ld32(st_tm + 32 * ch, sv);
                         tmem_ld32(dpt_tm + 32 * ch, dv);
-                        tmem_ld_wait();
+                        tmem_ld_wait_regs(sv);
+                        tmem_regs_fence(dv);
                         uint32_t pp[16], pd[16];
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
@@ -798,14 +837,19 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                                 const float4 a = cb[2 * c];
                                 const float4 b2 = cb[2 * c + 1];
                                 const int dist = delta0 + c - t;
-                                const float wv = biased ? run[c] : 0.0f;
-                                const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
                                 const bool vis = key_ok && dist >= 0 && i0 + c < p.T && (!edge || p.window <= 0 || dist < p.window);
+                                float wv = 0.0f;
+                                if (NCOPY > 0) {
+                                    if (biased) wv = run[c];
+                                } else if (biased && vis && dist < p.R) {
+                                    wv = __ldg(cstep + c * cstride - (c & 7));
+                                }
+                                const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
                                 const float pv = vis ? ex2_approx(x) : 0.0f;
                                 const float dl = pv * (__uint_as_float(dv[e + k]) - a.w);
                                 pr[k] = pv;
                                 dsv[k] = dl * b2.x;
-                                if (biased) {
+                                if (NCOPY > 0 && biased) {
                                     const float g = (dist >= 0 && dist < p.R) ? dl * b2.y : 0.0f;
                                     const float up = __shfl_up_sync(0xffffffffu, zdw, 1);
                                     zdw = g + (lane > 0 ? up : 0.0f);
@@ -817,12 +861,16 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                         }
                         tmem_st16(st_tm + 16 * ch + 32 * half, pp);
                         tmem_st16(dpt_tm + 16 * ch + 32 * half, pd);
+                        // pp and pd are this loop iteration's registers: wait before reuse.
+                        tmem_st_wait();
+                        tmem_regs_keep16(pp);
+                        tmem_regs_keep16(pd);
                     }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->pd_ready);
-                    if (biased) {
+                    if (NCOPY > 0 && biased) {
                         // Lane 31's sums: distance delta0 + c - (32 w + 31) at column c.
                         const int dbase = delta0 - ((t & ~31) + 31);
 #pragma unroll
@@ -839,7 +887,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (!ok) break;
                 // This head's table gradient from this key tile, into the output.
                 if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
-                for (int x = threadIdx.x; x < p.R; x += kBkRowWarps * 32)
+                for (int x = threadIdx.x; NCOPY > 0 && x < p.R; x += kBkRowWarps * 32)
                     if (dw_s[x] != 0.0f) atomicAdd(bp.dw + static_cast<size_t>(h) * p.R + x, dw_s[x]);
             }
             if (!ok) break;
@@ -852,7 +900,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 uint32_t a[32], b[32];
                 tmem_ld32(dk_tm + c, a);
                 tmem_ld32(dv_tm + c, b);
-                tmem_ld_wait();
+                tmem_ld_wait_regs(a);
+                tmem_regs_fence(b);
                 if (key_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
@@ -897,11 +946,11 @@ cudaError_t launch_bq(const CUtensorMap& tq, const CUtensorMap& tdo, const CUten
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, int NCOPY>
 cudaError_t launch_bk(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk, const CUtensorMap& tv,
                       const PrefillParams& p, const BwdTcParams& bp, int grid, cudaStream_t stream) {
-    auto kern = bwd_dkv_sm100_kernel<D, 1>;
-    const int smem = std::max(bk_smem_bytes(D, p.R, 1), 120 * 1024);
+    auto kern = bwd_dkv_sm100_kernel<D, NCOPY>;
+    const int smem = std::max(bk_smem_bytes(D, p.R, NCOPY), 120 * 1024);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kBkThreads, smem, stream>>>(tq, tdo, tk, tv, p, bp);
@@ -917,15 +966,128 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const C
                                                                                  p_dq.B, p_dq.T, p_dq.Hq);
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
+    const int g_dq = std::min(grid, p_dq.total_items), g_dkv = std::min(grid, p_dkv.total_items);
+    if (bp.curves != nullptr) {
+        // The bank form: biases from the per-row curves, dL/dcurve in place of dr and dw.
+        const cudaError_t e = launch_bq<D, 0>(tq, tdo, tk, tv, p_dq, bp, g_dq, stream);
+        if (e != cudaSuccess) return e;
+        return launch_bk<D, 0>(tq, tdo, tk, tv, p_dkv, bp, g_dkv, stream);
+    }
     const int nc = bq_copies<D>(p_dq.R);
-    cudaError_t e = nc == 4   ? launch_bq<D, 4>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)
-                    : nc == 2 ? launch_bq<D, 2>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream)
-                              : launch_bq<D, 1>(tq, tdo, tk, tv, p_dq, bp, std::min(grid, p_dq.total_items), stream);
+    cudaError_t e = nc == 4   ? launch_bq<D, 4>(tq, tdo, tk, tv, p_dq, bp, g_dq, stream)
+                    : nc == 2 ? launch_bq<D, 2>(tq, tdo, tk, tv, p_dq, bp, g_dq, stream)
+                              : launch_bq<D, 1>(tq, tdo, tk, tv, p_dq, bp, g_dq, stream);
     if (e != cudaSuccess) return e;
-    return launch_bk<D>(tq, tdo, tk, tv, p_dkv, bp, std::min(grid, p_dkv.total_items), stream);
+    return launch_bk<D, 1>(tq, tdo, tk, tv, p_dkv, bp, g_dkv, stream);
+}
+
+// ------------------------------------------------------------ bank-form gradients
+// From dcv[row, d] = tau_i dl(i, i-d) (the dQ kernel's output, padded rows of S floats,
+// row = (b * T + i) * Hq + h, distance d at 7 - (i & 7) + d):
+//   drs[row, c]     = sum_d dcv[row, d] proj[hp, c, d]
+//   dproj[hp, c, d] = sum over the rows of head group hp of rs[row, c] dcv[row, d]
+// (the chain rule through curve = sum_c rs[c] proj[c, :], "Thinking Machines dropped
+// RoPE", recipe step 2).
+constexpr int kDrsRows = 128;    // rows of one (b, h) per block, a thread each
+constexpr int kDrsChunk = 64;    // distances of proj staged per pass
+constexpr int kDprojRows = 512;  // rows of one (b, h) per block
+constexpr int kDprojThreads = 256;
+
+__global__ void __launch_bounds__(kDrsRows) bank_drs_kernel(const float* __restrict__ proj, const float* __restrict__ dcv,
+                                                            float* __restrict__ drs, int T, int Hq, int C,
+                                                            int proj_heads, int R, int S) {
+    __shared__ __align__(16) float pj[kDrsChunk][kMaxBankC];   // proj[hp, c, d0 + x] at [x][c]
+    const int iblocks = (T + kDrsRows - 1) / kDrsRows;
+    const int ib = static_cast<int>(blockIdx.x) % iblocks;
+    const int bh = static_cast<int>(blockIdx.x) / iblocks;
+    const int h = bh % Hq, b = bh / Hq;
+    const int i = ib * kDrsRows + static_cast<int>(threadIdx.x);
+    const bool ok = i < T;
+    const size_t row = (static_cast<size_t>(b) * T + (ok ? i : 0)) * Hq + h;
+    const float* dc = dcv + row * S + (7 - (i & 7));
+    const float* pr = proj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
+    float acc[kMaxBankC];
+#pragma unroll
+    for (int c = 0; c < kMaxBankC; ++c) acc[c] = 0.0f;
+    for (int d0 = 0; d0 < R; d0 += kDrsChunk) {
+        __syncthreads();
+        for (int x = threadIdx.x; x < kDrsChunk * kMaxBankC; x += kDrsRows) {
+            const int c = x / kDrsChunk, dd = x % kDrsChunk;
+            pj[dd][c] = (c < C && d0 + dd < R) ? __ldg(pr + static_cast<size_t>(c) * R + d0 + dd) : 0.0f;
+        }
+        __syncthreads();
+        if (!ok) continue;
+        const int dn = min(kDrsChunk, R - d0);
+#pragma unroll 4
+        for (int x = 0; x < dn; ++x) {
+            const float v = __ldg(dc + d0 + x);
+#pragma unroll
+            for (int c = 0; c < kMaxBankC; c += 4) {
+                const float4 q = *reinterpret_cast<const float4*>(&pj[x][c]);
+                acc[c] = fmaf(v, q.x, acc[c]), acc[c + 1] = fmaf(v, q.y, acc[c + 1]);
+                acc[c + 2] = fmaf(v, q.z, acc[c + 2]), acc[c + 3] = fmaf(v, q.w, acc[c + 3]);
+            }
+        }
+    }
+    if (ok)
+        for (int c = 0; c < C; ++c) drs[row * C + c] = acc[c];
+}
+
+__global__ void __launch_bounds__(kDprojThreads) bank_dproj_kernel(const float* __restrict__ rs,
+                                                                   const float* __restrict__ dcv,
+                                                                   float* __restrict__ dproj, int T, int Hq, int C,
+                                                                   int proj_heads, int R, int S) {
+    __shared__ __align__(16) float rsm[kDprojRows][kMaxBankC];
+    const int iblocks = (T + kDprojRows - 1) / kDprojRows;
+    const int ib = static_cast<int>(blockIdx.x) % iblocks;
+    const int bh = static_cast<int>(blockIdx.x) / iblocks;
+    const int h = bh % Hq, b = bh / Hq;
+    const int i0 = ib * kDprojRows;
+    for (int x = threadIdx.x; x < kDprojRows * kMaxBankC; x += kDprojThreads) {
+        const int r = x / kMaxBankC, c = x % kMaxBankC;
+        const int i = i0 + r;
+        rsm[r][c] = (i < T && c < C) ? __ldg(rs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C + c) : 0.0f;
+    }
+    __syncthreads();
+    const int nrows = min(kDprojRows, T - i0);
+    const size_t row_step = static_cast<size_t>(Hq) * S;     // floats between rows i and i + 1
+    const float* base = dcv + ((static_cast<size_t>(b) * T + i0) * Hq + h) * S;
+    float* out = dproj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
+    for (int d = threadIdx.x; d < R; d += kDprojThreads) {
+        float acc[kMaxBankC];
+#pragma unroll
+        for (int c = 0; c < kMaxBankC; ++c) acc[c] = 0.0f;
+#pragma unroll 4
+        for (int r = 0; r < nrows; ++r) {
+            const float v = __ldg(base + r * row_step + (7 - ((i0 + r) & 7)) + d);
+#pragma unroll
+            for (int c = 0; c < kMaxBankC; c += 4) {
+                const float4 q = *reinterpret_cast<const float4*>(&rsm[r][c]);
+                acc[c] = fmaf(v, q.x, acc[c]), acc[c + 1] = fmaf(v, q.y, acc[c + 1]);
+                acc[c + 2] = fmaf(v, q.z, acc[c + 2]), acc[c + 3] = fmaf(v, q.w, acc[c + 3]);
+            }
+        }
+        for (int c = 0; c < C; ++c) atomicAdd(out + static_cast<size_t>(c) * R + d, acc[c]);
+    }
 }
 
 }  // namespace
+
+bool backward_bank_tc_supported(int d) { return d == 128 || d == 64; }
+
+cudaError_t launch_bank_grads(const float* rs, const float* proj, const float* dcv, float* drs, float* dproj, int B,
+                              int T, int Hq, int C, int proj_heads, int R, int S, cudaStream_t stream) {
+    if (B < 1 || T < 1 || R < 1) return cudaSuccess;
+    const long long bh = static_cast<long long>(B) * Hq;
+    const long long n1 = bh * ((T + kDrsRows - 1) / kDrsRows), n2 = bh * ((T + kDprojRows - 1) / kDprojRows);
+    if (n1 > INT32_MAX || n2 > INT32_MAX) return cudaErrorInvalidValue;
+    bank_drs_kernel<<<static_cast<unsigned>(n1), kDrsRows, 0, stream>>>(proj, dcv, drs, T, Hq, C, proj_heads, R, S);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bank_dproj_kernel<<<static_cast<unsigned>(n2), kDprojThreads, 0, stream>>>(rs, dcv, dproj, T, Hq, C, proj_heads, R,
+                                                                               S);
+    return cudaGetLastError();
+}
 
 bool backward_tc_supported(int d, int R) {
     if (d == 128) return bq_copies<128>(R) > 0 && bk_smem_bytes(128, R, 1) <= kMaxDynSmem;

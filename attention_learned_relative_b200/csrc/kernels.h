@@ -76,8 +76,20 @@ struct BwdTcParams {
     float* dv;                  // [B, T, Hkv, d]
     float* dw;                  // [Hq, R], zeroed by the caller, accumulated atomically
     float scale;
+    // Shared-bank form (curves != nullptr): the bias of row (b, i, h) at distance d is
+    // curves[row * curve_stride + pad + d] (the padded layout of launch_bank_rows), and
+    // the dQ kernel writes dL/dcurve, tau_i * dl(i, i-d), to dcv in the same layout
+    // (zeroed by the caller) in place of dr and dw.
+    const float* curves;
+    float* dcv;
+    int curve_stride;
 };
 bool backward_tc_supported(int d, int R);
+bool backward_bank_tc_supported(int d);
+// dL/drs[row, c] = sum_d dcv[row, d] proj[hp, c, d] and dL/dproj[hp, c, d] += sum over
+// the rows of head group hp of rs[row, c] dcv[row, d] (dproj zeroed by the caller).
+cudaError_t launch_bank_grads(const float* rs, const float* proj, const float* dcv, float* drs, float* dproj, int B,
+                              int T, int Hq, int C, int proj_heads, int R, int S, cudaStream_t stream);
 cudaError_t launch_backward_sm100(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
                                   const BwdTcParams& bp, int d, int grid, cudaStream_t stream);

@@ -682,7 +682,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t sr[kBN];
 #pragma unroll
                     for (int c = 0; c < kBN; c += 32) tmem_ld32(s_tm + c, sr + c);
-                    tmem_ld_wait();
+                    tmem_ld_wait_regs(sr);
+#pragma unroll
+                    for (int c = 32; c < kBN; c += 32) tmem_regs_fence(sr + c);
                     float s[kBN];
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
@@ -779,10 +781,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < D; c += 32) {
                             tmem_ld32(o_tm + c, ob);
-                            tmem_ld_wait();
+                            tmem_ld_wait_regs(ob);
 #pragma unroll
                             for (int e = 0; e < 32; ++e) ob[e] = __float_as_uint(__uint_as_float(ob[e]) * alpha);
                             tmem_st32(o_tm + c, ob);
+                            tmem_st_wait();   // ob is refilled by the next chunk
+                            tmem_regs_keep16(ob);
+                            tmem_regs_keep16(ob + 16);
                         }
                         tmem_st_wait();
                     }
@@ -791,6 +796,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st32(s_tm, pk);
                 tmem_st32(s_tm + 32, pk + 32);
                 tmem_st_wait();
+#pragma unroll
+                for (int c = 0; c < kBN / 2; c += 16) tmem_regs_keep16(pk + c);
                 tc_fence_before();
                 // One arrival per warp, once every lane's P is in tensor memory.
                 __syncwarp();
@@ -812,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < D; c += 32) {
                 uint32_t ob[32];
                 tmem_ld32(o_tm + c, ob);
-                tmem_ld_wait();
+                tmem_ld_wait_regs(ob);
                 uint32_t packed[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)

@@ -587,7 +587,7 @@ namespace {
 int bwd_tc_impl(const void* q, const void* k, const void* v, const float* r, const float* w, const void* o,
                 const float* lse, const void* dout, float* dq, float* dk, float* dv, float* dr, float* dw, int B,
                 int T, int Hq, int Hkv, int d, int window, int R, float scale, int temp_n0, float* dvec, int sms,
-                cudaStream_t st) {
+                cudaStream_t st, const float* curves = nullptr, float* dcv = nullptr, int curve_stride = 0) {
     int rc;
     CUtensorMap tq, tdo, tk, tv;
     if ((rc = make_map(&tq, q, B, T, Hq, d, 128)) != RELBIAS_OK) return rc;
@@ -631,7 +631,10 @@ int bwd_tc_impl(const void* q, const void* k, const void* v, const float* r, con
     bp.dv = dv;
     bp.dw = dw;
     bp.scale = scale;
-    if (R > 0) {
+    bp.curves = curves;
+    bp.dcv = dcv;
+    bp.curve_stride = curve_stride;
+    if (R > 0 && dw != nullptr) {
         const cudaError_t e = cudaMemsetAsync(dw, 0, static_cast<size_t>(Hq) * R * sizeof(float), st);
         if (e != cudaSuccess) return cuda_fail(e, "clearing dw");
     }
@@ -681,6 +684,70 @@ extern "C" int relbias_attn_bwd(const void* q, const void* k, const void* v, con
                                           static_cast<float*>(workspace), B, T, Hq, Hkv, window > 0 ? window : 0, R,
                                           scale, temp_n0 > 1 ? temp_n0 : 0, st);
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "backward launch");
+}
+
+namespace {
+// The bank form's backward workspace: D_i [B, Hq, T], then the per-row curves and
+// their gradient, each [B, T, Hq, S] floats (S = prefill_bank_curve_stride(R)), each
+// part starting on a 256-byte boundary.
+size_t bwd_bank_part(size_t bytes) { return (bytes + 255) / 256 * 256; }
+}  // namespace
+
+extern "C" size_t relbias_attn_bwd_bank_workspace_size(int B, int T, int Hq, int R) {
+    if (B < 0 || T < 0 || Hq < 1 || R < 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * T * Hq;
+    return bwd_bank_part(rows * sizeof(float)) + 2 * bwd_bank_part(rows * prefill_bank_curve_stride(R) * sizeof(float));
+}
+
+extern "C" int relbias_attn_bwd_bank(const void* q, const void* k, const void* v, const float* rs, const float* proj,
+                                     const void* o, const float* lse, const void* dout, float* dq, float* dk,
+                                     float* dv, float* drs, float* dproj, int B, int T, int Hq, int Hkv, int d, int C,
+                                     int proj_heads, int window, int R, float scale, int temp_n0, int dtype,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+    t_err.clear();
+    int rc = check_common(B, T, Hq, Hkv, d, R, scale, proj);
+    if (rc != RELBIAS_OK) return rc;
+    if ((rc = check_bank(C, proj_heads, Hq)) != RELBIAS_OK) return rc;
+    if (dtype != RELBIAS_BF16 && dtype != RELBIAS_FP32) return fail(RELBIAS_ERR_ARG, "unknown dtype %d", dtype);
+    if (B == 0 || T == 0) return RELBIAS_OK;
+    if (dtype != RELBIAS_BF16 || !backward_bank_tc_supported(d))
+        return fail(RELBIAS_ERR_UNSUPPORTED, "the bank-form backward runs bf16 with d in {64, 128}");
+    if (R < 1) return fail(RELBIAS_ERR_UNSUPPORTED, "the bank-form backward needs R >= 1 (R = 0 has no bias)");
+    if (R > 2048) return fail(RELBIAS_ERR_UNSUPPORTED, "the bank-form backward supports R <= 2048, got %d", R);
+    if (static_cast<long long>(B) * T * Hq > INT32_MAX)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "B * T * Hq must stay below 2^31");
+    if (!q || !k || !v || !rs || !proj || !o || !lse || !dout || !dq || !dk || !dv || !drs || !dproj || !workspace)
+        return fail(RELBIAS_ERR_ARG, "no pointer argument may be null");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(RELBIAS_ERR_ARG, "q, k, v, o, dout, dq, dk and dv must be 16-byte aligned, workspace 256-byte");
+    if (!aligned4(rs) || !aligned4(proj) || !aligned4(lse) || !aligned4(drs) || !aligned4(dproj))
+        return fail(RELBIAS_ERR_ARG, "rs, proj, lse, drs and dproj must be 4-byte aligned");
+    const size_t need = relbias_attn_bwd_bank_workspace_size(B, T, Hq, R);
+    if (ws_bytes < need)
+        return fail(RELBIAS_ERR_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", ws_bytes, need);
+    DeviceInfo dev;
+    if ((rc = device_info(dev)) != RELBIAS_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0)
+        return fail(RELBIAS_ERR_UNSUPPORTED, "the bank-form backward needs an sm_100 device");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t rows = static_cast<size_t>(B) * T * Hq;
+    const int S = prefill_bank_curve_stride(R);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* dvec = reinterpret_cast<float*>(ws);
+    float* curves = reinterpret_cast<float*>(ws + bwd_bank_part(rows * sizeof(float)));
+    float* dcv = reinterpret_cast<float*>(ws + bwd_bank_part(rows * sizeof(float)) +
+                                          bwd_bank_part(rows * S * sizeof(float)));
+    cudaError_t e = launch_bank_rows(rs, proj, curves, B, T, Hq, 0, C, proj_heads, R, st);
+    if (e != cudaSuccess) return cuda_fail(e, "bank curve launch");
+    if ((e = cudaMemsetAsync(dcv, 0, rows * S * sizeof(float), st)) != cudaSuccess) return cuda_fail(e, "clearing dcv");
+    if ((e = cudaMemsetAsync(dproj, 0, static_cast<size_t>(proj_heads) * C * R * sizeof(float), st)) != cudaSuccess)
+        return cuda_fail(e, "clearing dproj");
+    rc = bwd_tc_impl(q, k, v, rs, proj, o, lse, dout, dq, dk, dv, nullptr, nullptr, B, T, Hq, Hkv, d, window, R,
+                     scale, temp_n0, dvec, dev.sms, st, curves, dcv, S);
+    if (rc != RELBIAS_OK) return rc;
+    e = launch_bank_grads(rs, proj, dcv, drs, dproj, B, T, Hq, C, proj_heads, R, S, st);
+    return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "bank gradient launch");
 }
 
 extern "C" const char* relbias_last_error(void) { return t_err.c_str(); }

@@ -52,6 +52,8 @@ SIGNATURES = {
                                       _I, _VP, _SZ, _VP]),
     "relbias_attn_bwd_workspace_size": (_SZ, [_I, _I, _I]),
     "relbias_attn_bwd": (_I, [_VP] * 13 + [_I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
+    "relbias_attn_bwd_bank_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "relbias_attn_bwd_bank": (_I, [_VP] * 13 + [_I] * 9 + [_F, _I, _I, _VP, _SZ, _VP]),
     "relbias_last_error": (ctypes.c_char_p, []),
     "relbias_device_status": (_I, [_I]),
     "relbias_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
@@ -425,6 +427,44 @@ def attn_bwd(q, k, v, r, w, o, lse, dout, window: int, R: int, scale: float | No
     _check(rc)
     return g
 
+
+
+def attn_bwd_bank(q, k, v, rs, proj, o, lse, dout, window: int, R: int, scale: float | None = None, stream=None,
+                  temp_n0: int = 0, workspace=None, grads=None):
+    """Backward pass of attn_fwd_bank (bf16, d in {64, 128}).  rs [B,T,Hq,C] and proj
+    [1 or Hq, C, R] fp32, the rest as attn_bwd.  Returns a dict of fp32 gradients dq,
+    dk, dv, drs (shaped like rs) and dproj (shaped like proj), written into `grads`
+    when a dict of such tensors is given."""
+    _need(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,T,Hq,d], k/v [B,T,Hkv,d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(o.shape == q.shape and dout.shape == q.shape, "o and dout must have q's shape")
+    _need(q.dtype == k.dtype == v.dtype == o.dtype == dout.dtype, "q, k, v, o, dout must share a dtype")
+    _need(rs.dim() == 4 and rs.shape[:3] == (B, T, Hq) and rs.dtype == torch.float32, "rs must be fp32 [B,T,Hq,C]")
+    C = int(rs.shape[3])
+    proj_heads = _bank_shape(proj, C, Hq, R)
+    _need(lse.shape == (B, Hq, T) and lse.dtype == torch.float32, "lse must be fp32 [B,Hq,T]")
+    for t in (q, k, v, rs, proj, o, lse, dout, workspace):
+        _need(t is None or (t.is_cuda and t.is_contiguous()), "tensors must be contiguous CUDA tensors")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = grads if grads is not None else {
+        "dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32), "dv": torch.empty(v.shape, **f32),
+        "drs": torch.empty(rs.shape, **f32), "dproj": torch.empty(proj.shape, **f32)}
+    for name, like in (("dq", q), ("dk", k), ("dv", v), ("drs", rs), ("dproj", proj)):
+        _need(g[name].shape == like.shape and g[name].dtype == torch.float32 and g[name].is_contiguous(),
+              "%s must be a contiguous fp32 tensor of shape %s" % (name, tuple(like.shape)))
+    need = int(lib().relbias_attn_bwd_bank_workspace_size(B, T, Hq, R))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = lib().relbias_attn_bwd_bank(_ptr(q), _ptr(k), _ptr(v), _ptr(rs), _ptr(proj), _ptr(o), _ptr(lse), _ptr(dout),
+                                     _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["drs"]), _ptr(g["dproj"]),
+                                     B, T, Hq, Hkv, d, C, proj_heads, int(window), int(R), float(scale), int(temp_n0),
+                                     _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
+    _check(rc)
+    return g
 
 def device_status(reset: bool = True) -> int:
     """Synchronise and return the kernels' status bits (RELBIAS_STATUS_*)."""

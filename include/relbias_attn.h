@@ -324,8 +324,11 @@ RELBIAS_API int relbias_attn_decode_bank(const void* q, const void* k_cache, con
  *   workspace: at least relbias_attn_bwd_workspace_size(B, T, Hq) bytes of
  *     caller-owned device scratch (D_i per row), 16-byte aligned.
  * o and lse must be the forward's outputs for the same inputs.  dtype
- * RELBIAS_BF16 or RELBIAS_FP32 (fp32 arithmetic on CUDA cores either way);
- * d in {32, 64, 128, 256}; R <= 32768; other rules as for relbias_attn_fwd.
+ * RELBIAS_BF16 or RELBIAS_FP32.  bf16 with d in {64, 128} on sm_100 runs on the
+ * tensor cores (bf16 products of the recomputed P and dS, fp32 accumulation; dr and
+ * dw are summed with fp32 atomics, so dw is not bitwise repeatable); fp32 and other
+ * head sizes run in fp32 on CUDA cores.  d in {32, 64, 128, 256}; R <= 32768; other
+ * rules as for relbias_attn_fwd.
  */
 RELBIAS_API size_t relbias_attn_bwd_workspace_size(int B, int T, int Hq);
 RELBIAS_API int relbias_attn_bwd(const void* q, const void* k, const void* v,
@@ -333,6 +336,35 @@ RELBIAS_API int relbias_attn_bwd(const void* q, const void* k, const void* v,
                      const void* o, const float* lse, const void* dout,
                      float* dq, float* dk, float* dv, float* dr, float* dw,
                      int B, int T, int Hq, int Hkv, int d,
+                     int window, int R, float scale, int temp_n0,
+                     int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Backward pass of relbias_attn_fwd_bank (the shared-bank bias of the essay's
+ * recipe steps 1-2, curve_i = sum_c rs[b,i,h,c] * proj[h', c, :]).  With
+ * dcurve_i[d] = tau_i * dl_(i, i-d) for 0 <= d < R (the gradient of row i's curve):
+ *   drs[b,i,h,c]   = sum_d dcurve_i[d] * proj[h', c, d]
+ *   dproj[h', c, d] = sum over the rows (b, i, h) that use bank h' of rs[b,i,h,c] * dcurve_i[d]
+ * and dq, dk, dv as for relbias_attn_bwd.
+ *
+ *   rs [B, T, Hq, C], proj [proj_heads, C, R] fp32 (1 <= C <= 16, proj_heads 1 or Hq)
+ *   drs [B, T, Hq, C], dproj [proj_heads, C, R]: fp32 outputs, overwritten
+ *   workspace: at least relbias_attn_bwd_bank_workspace_size(B, T, Hq, R) bytes of
+ *     caller-owned device scratch, 256-byte aligned: D_i per row, then each row's
+ *     curve and its gradient (two padded fp32 rows of R + 14..21 floats per (b, i, h)).
+ * Runs the curve kernel of relbias_attn_fwd_bank, the tensor-core dQ and dK/dV
+ * kernels reading each row's curve in place of r * w (the dQ kernel writing
+ * dcurve), then two reductions for drs and dproj.  dproj is summed with fp32 atomics
+ * and is not bitwise repeatable.  RELBIAS_BF16 with d in {64, 128} on sm_100 only
+ * (RELBIAS_ERR_UNSUPPORTED otherwise); 1 <= R <= 2048; B * T * Hq < 2^31; other
+ * rules as for relbias_attn_bwd.
+ */
+RELBIAS_API size_t relbias_attn_bwd_bank_workspace_size(int B, int T, int Hq, int R);
+RELBIAS_API int relbias_attn_bwd_bank(const void* q, const void* k, const void* v,
+                     const float* rs, const float* proj,
+                     const void* o, const float* lse, const void* dout,
+                     float* dq, float* dk, float* dv, float* drs, float* dproj,
+                     int B, int T, int Hq, int Hkv, int d, int C, int proj_heads,
                      int window, int R, float scale, int temp_n0,
                      int dtype, void* workspace, size_t ws_bytes, void* stream);
 

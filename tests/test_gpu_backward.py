@@ -109,3 +109,54 @@ def test_backward_is_deterministic_except_dw(dtype):
     for name in ("dq", "dk", "dv", "dr"):
         assert torch.equal(g1[name], g2[name]), name
     assert (g1["dw"] - g2["dw"]).abs().max().item() <= 1e-5 * g1["dw"].abs().max().item()
+
+
+# The shared-bank form (relbias_attn_bwd_bank): bf16, d in {64, 128}.
+BANK_CASES = [
+    # B, T,   Hq, Hkv, d,   window, R,   C,  proj_heads, temp_n0
+    (1, 300, 8, 2, 128, 0, 256, 16, 1, 0),       # the essay's 16-function bank, shared by the layer
+    (1, 640, 8, 2, 128, 512, 512, 16, 8, 0),     # a bank per head, the local layer's window
+    (2, 200, 6, 3, 64, 0, 150, 5, 1, 100),       # d = 64, odd group, R not a multiple of 8, temperature
+    (1, 129, 4, 2, 128, 64, 30, 3, 4, 0),        # one tile plus one row, window < tile
+]
+
+
+def _bank_inputs(B, T, Hq, Hkv, d, R, C, proj_heads, seed):
+    x = _inputs(torch.bfloat16, B, T, Hq, Hkv, d, R, seed)
+    x["rs"] = synth.normal((B, T, Hq, C), seed, "rs", std=1.0 / math.sqrt(C), device="cuda")
+    x["proj"] = synth.normal((proj_heads, C, R), seed, "proj", std=0.5, device="cuda")
+    return x
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,d,window,R,C,proj_heads,temp_n0", BANK_CASES)
+def test_backward_bank_parity(B, T, Hq, Hkv, d, window, R, C, proj_heads, temp_n0):
+    """Gradients of the bank form (dq, dk, dv, drs, dproj) against the oracle's."""
+    x = _bank_inputs(B, T, Hq, Hkv, d, R, C, proj_heads, seed=T + C + R)
+    scale = 1.0 / math.sqrt(d)
+    o_ref, lse_ref = O.attn_prefill(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["rs"].cpu(), x["proj"].cpu(),
+                                    window, R, scale, temp_n0=temp_n0)
+    o = torch.as_tensor(o_ref).to(torch.bfloat16).cuda()
+    lse = torch.as_tensor(lse_ref).float().cuda()
+    g = ops.attn_bwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], o, lse, x["dout"], window, R, scale,
+                          temp_n0=temp_n0)
+    torch.cuda.synchronize()
+    ref = O.attn_backward(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), x["rs"].cpu(), x["proj"].cpu(),
+                          x["dout"].cpu(), window, R, scale, temp_n0=temp_n0)
+    _check({"dq": g["dq"], "dk": g["dk"], "dv": g["dv"], "dr": g["drs"], "dw": g["dproj"]}, ref, 1e-2,
+           "bank backward %s" % ((B, T, Hq, Hkv, d, window, R, C, proj_heads, temp_n0),))
+
+
+def test_backward_bank_of_one_function_per_head_matches_rank1():
+    """C = 1 with a bank per head is the rank-1 form: the same gradients (drs = dr,
+    dproj = dw) up to the order of the fp32 sums."""
+    B, T, Hq, Hkv, d, window, R = 1, 400, 8, 2, 128, 256, 256
+    x = _inputs(torch.bfloat16, B, T, Hq, Hkv, d, R, seed=21)
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], window, R, lse=lse)
+    g1 = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], window, R)
+    g2 = ops.attn_bwd_bank(x["q"], x["k"], x["v"], x["r"][..., None].contiguous(), x["w"][:, None, :].contiguous(),
+                           o, lse, x["dout"], window, R)
+    torch.cuda.synchronize()
+    for a, b in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dr", "drs"), ("dw", "dproj")):
+        u, w = g1[a].reshape(-1), g2[b].reshape(-1)
+        assert (u - w).abs().max().item() <= 1e-4 * u.abs().max().item() + 1e-7, a

@@ -203,3 +203,22 @@ def test_bank_prefill_writes_stay_inside(B, T, Hq, Hkv, d, window, R, C, proj_he
     o.check("o")
     lse.check("lse")
     ws.check("workspace", fully_written=False)
+
+
+def test_bank_backward_writes_stay_inside():
+    B, T, Hq, Hkv, d, R, C = 1, 200, 6, 2, 64, 77, 5
+    x = _x(B, T, Hq, Hkv, d, R, seed=31)
+    rs = synth.normal((B, T, Hq, C), 31, "rs", std=0.4, device="cuda")
+    proj = synth.normal((1, C, R), 31, "proj", std=0.5, device="cuda")
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    o = ops.attn_fwd_bank(x["q"], x["k"], x["v"], rs, proj, 64, R, 0.125, lse=lse)
+    dout = synth.normal((B, T, Hq, d), 3, "bank", dtype=torch.bfloat16, device="cuda")
+    g = {"dq": Guarded((B, T, Hq, d), torch.float32), "dk": Guarded((B, T, Hkv, d), torch.float32),
+         "dv": Guarded((B, T, Hkv, d), torch.float32), "drs": Guarded((B, T, Hq, C), torch.float32),
+         "dproj": Guarded((1, C, R), torch.float32)}
+    ws = Guarded((int(ops.lib().relbias_attn_bwd_bank_workspace_size(B, T, Hq, R)),), torch.uint8)
+    ops.attn_bwd_bank(x["q"], x["k"], x["v"], rs, proj, o, lse, dout, 64, R, 0.125, workspace=ws.t,
+                      grads={n: gb.t for n, gb in g.items()})
+    for n, gb in g.items():
+        gb.check(n)
+    ws.check("workspace", fully_written=False)
