@@ -98,6 +98,9 @@ WORKLOADS = {
         # The backward pass of the local-layer prefill (the pages train the model).
         Workload("local_backward_bf16", B=2, T=8192, Hq=32, Hkv=4, d=128, window=512, R=512,
                  seed=1, dtype="bf16", backward=True),
+        # The same backward with the shared-bank bias (16 functions shared by all heads).
+        Workload("local_backward_bank_bf16", B=2, T=8192, Hq=32, Hkv=4, d=128, window=512, R=512,
+                 seed=1, dtype="bf16", backward=True, bank_C=16),
     ]
 }
 

@@ -207,9 +207,11 @@ def launches_per_step(wl) -> int:
     """Kernels of this library one step launches."""
     if wl.decode:
         return 3 if wl.bank_C > 0 else 2       # (bank curves), split-KV, combine
+    if wl.backward:                            # D_i, dq, dk/dv (+ bank curves, drs, dproj)
+        return 6 if wl.bank_C > 0 else 3
     if wl.bank_C > 0:
         return 2                               # bank curves, prefill
-    return 2 if wl.backward else 1             # dq + dk/dv kernels, or the one prefill kernel
+    return 1                                   # the one prefill kernel
 
 
 def workload_config(wl, world, l2_note):
@@ -217,7 +219,8 @@ def workload_config(wl, world, l2_note):
             "window": wl.window, "R": wl.R, "global_batch": wl.B * world,
             **({"page_size": wl.page_size, "pages": "shuffled pool"} if wl.page_size > 0 else {}),
             **({"bias": "shared bank, C=%d functions" % wl.bank_C} if wl.bank_C > 0 else {}),
-            **({"pass": "backward (dq, dk, dv, dr, dw)"} if wl.backward else {}),
+            **({"pass": "backward (dq, dk, dv, %s)" % ("drs, dproj" if wl.bank_C > 0 else "dr, dw")}
+               if wl.backward else {}),
             "parallelism": "dp%d (batch shards, no collective)" % world,
             "l2": l2_note}
 
@@ -245,11 +248,17 @@ def make_sets(wl, nsets, device, shared=None):
             # The forward's O and LSE are inputs of the backward: computed once, untimed.
             from attention_learned_relative_b200 import ops
             x["lse"] = torch.empty(wl.B, wl.Hq, wl.T, dtype=torch.float32, device=device)
-            x["o"] = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, lse=x["lse"])
             f32 = dict(dtype=torch.float32, device=device)
             x["g"] = {"dq": torch.empty(x["q"].shape, **f32), "dk": torch.empty(x["k"].shape, **f32),
-                      "dv": torch.empty(x["v"].shape, **f32), "dr": torch.empty(x["r"].shape, **f32),
-                      "dw": torch.empty(wl.Hq, wl.R, **f32)}
+                      "dv": torch.empty(x["v"].shape, **f32)}
+            if wl.bank_C > 0:
+                x["o"] = ops.attn_fwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], wl.window, wl.R, wl.scale,
+                                           lse=x["lse"])
+                x["g"].update(drs=torch.empty(x["rs"].shape, **f32), dproj=torch.empty(x["proj"].shape, **f32))
+            else:
+                x["o"] = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale,
+                                      lse=x["lse"])
+                x["g"].update(dr=torch.empty(x["r"].shape, **f32), dw=torch.empty(wl.Hq, wl.R, **f32))
         else:
             x["o"] = torch.empty_like(x["q"])
             x["lse"] = torch.empty(wl.B, wl.Hq, wl.T, dtype=torch.float32, device=device)
@@ -271,6 +280,10 @@ def step_fn(wl, ops, workspace):
         def step(x, stream):
             ops.attn_decode(x["q"], x["k"], x["v"], x["r"], x["w"], wl.window, wl.R, wl.scale, out=x["o"],
                             lse=x["lse"], workspace=workspace, stream=stream)
+    elif wl.backward and wl.bank_C > 0:
+        def step(x, stream):
+            ops.attn_bwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], x["o"], x["lse"], x["dout"], wl.window,
+                              wl.R, wl.scale, stream=stream, workspace=workspace, grads=x["g"])
     elif wl.bank_C > 0:
         def step(x, stream):
             ops.attn_fwd_bank(x["q"], x["k"], x["v"], x["rs"], x["proj"], wl.window, wl.R, wl.scale, out=x["o"],
@@ -289,7 +302,7 @@ def step_fn(wl, ops, workspace):
 def step_outputs(wl, x):
     """The device tensors a step produces (read back to the host in the e2e measurement)."""
     if wl.backward:
-        return [x["g"][n] for n in ("dq", "dk", "dv", "dr", "dw")]
+        return [x["g"][n] for n in ("dq", "dk", "dv") + (("drs", "dproj") if wl.bank_C > 0 else ("dr", "dw"))]
     return [x["o"]]
 
 
@@ -335,9 +348,10 @@ def cpu_baseline(wl, x, budget_s):
         # The oracle's backward over a prefix of sequence 0 (all heads): causal, so the
         # prefix is a complete sub-problem.  Its length is sized to the time budget.
         def run(n):
-            args = [x[t][:1, :n].cpu() for t in ("q", "k", "v", "r")]
+            bias = ("rs", "proj") if wl.bank_C > 0 else ("r", "w")
+            args = [x[t][:1, :n].cpu() for t in ("q", "k", "v", bias[0])]
             t0 = time.perf_counter()
-            O.attn_backward(args[0], args[1], args[2], args[3], x["w"].cpu(), x["dout"][:1, :n].cpu(), wl.window,
+            O.attn_backward(args[0], args[1], args[2], args[3], x[bias[1]].cpu(), x["dout"][:1, :n].cpu(), wl.window,
                             wl.R, wl.scale)
             return time.perf_counter() - t0
 
@@ -399,7 +413,8 @@ def cpu_baseline(wl, x, budget_s):
 # Workloads the default run measures beside the headline one, each in its own timed
 # region, reported in the same JSON line under "per_config".
 PER_CONFIG = ["local_prefill_bank_bf16", "global_prefill_bf16", "global_long_prefill_bf16", "global_decode_bf16",
-              "global_decode_paged_bf16", "global_decode_bank_bf16", "local_backward_bf16"]
+              "global_decode_paged_bf16", "global_decode_bank_bf16", "local_backward_bf16",
+              "local_backward_bank_bf16"]
 
 
 def roofline_of(wl, ms_step, peaks, peaks_kind):
@@ -422,6 +437,8 @@ def roofline_of(wl, ms_step, peaks, peaks_kind):
     peak = float(peaks["bf16_tflops"]) if tensor else 148 * 128 * 2 * 1.965e9 / 1e12
     if wl.backward:
         kernel = "bwd_dq_sm100_kernel + bwd_dkv_sm100_kernel" if tensor else "bwd_dq_kernel + bwd_dkv_kernel"
+        if wl.bank_C > 0:
+            kernel = "bank_rows_kernel + " + kernel + " + bank_drs_kernel + bank_dproj_kernel"
     elif wl.dtype == "bf16":
         kernel = "bank_rows_kernel + prefill_bf16_sm100_kernel" if wl.bank_C > 0 else "prefill_bf16_sm100_kernel"
     else:
@@ -447,10 +464,13 @@ def measure(args, wl, ctx, steps_arg, e2e_on, cpu_budget, shared=None):
     wl_r, _ = rank_workload(wl, rank, world)
     sets = make_sets(wl_r, nsets, dev, shared)
     workspace = None
-    if wl.backward:
+    if wl.backward and wl.bank_C > 0:
+        workspace = torch.empty(max(256, ops.lib().relbias_attn_bwd_bank_workspace_size(wl.B, wl.T, wl.Hq, wl.R)),
+                                dtype=torch.uint8, device=dev)
+    elif wl.backward:
         workspace = torch.empty(max(16, ops.lib().relbias_attn_bwd_workspace_size(wl.B, wl.T, wl.Hq)),
                                 dtype=torch.uint8, device=dev)
-    if wl.bank_C > 0 and not wl.decode:
+    elif wl.bank_C > 0 and not wl.decode:
         nbytes = ops.fwd_bank_workspace_size(wl.B, wl.T, wl.Hq, wl.R,
                                              ops.RELBIAS_BF16 if wl.dtype == "bf16" else ops.RELBIAS_FP32)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
@@ -501,7 +521,7 @@ def measure(args, wl, ctx, steps_arg, e2e_on, cpu_budget, shared=None):
         if wl.decode:
             names_in = ["q", "rs"] if wl.bank_C > 0 else ["q", "r"]
         elif wl.backward:
-            names_in = ["q", "k", "v", "r", "w", "o", "lse", "dout"]
+            names_in = ["q", "k", "v"] + (["rs", "proj"] if wl.bank_C > 0 else ["r", "w"]) + ["o", "lse", "dout"]
         elif wl.bank_C > 0:
             names_in = ["q", "k", "v", "rs", "proj"]
         else:

@@ -160,3 +160,53 @@ def test_backward_bank_of_one_function_per_head_matches_rank1():
     for a, b in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dr", "drs"), ("dw", "dproj")):
         u, w = g1[a].reshape(-1), g2[b].reshape(-1)
         assert (u - w).abs().max().item() <= 1e-4 * u.abs().max().item() + 1e-7, a
+
+
+@pytest.mark.parametrize("bank", [False, True])
+def test_backward_full_size_local_layer_sampled(bank):
+    """The local-layer workload at full size (B=2, T=8192, Hq=32, Hkv=4, d=128, window =
+    R = 512, bf16), in the launch configuration the bench times.  A row's dq and dr
+    depend only on the 512 keys it sees, and a key's dk and dv only on the 512 rows that
+    see it, so the oracle over positions [i0 - 511, i0 + 64 + 511) of one sequence and
+    one key/value head (with its 8 query heads) gives exact references for rows
+    [i0, i0 + 64) (dq, dr: every key they see is in the slice) and
+    keys [i0, i0 + 64) (dk, dv: every row that sees them is in the slice, with all of
+    its own keys)."""
+    from attention_learned_relative_b200 import workloads
+    wl = workloads.WORKLOADS["local_backward_bf16"]
+    x = workloads.make_inputs(wl, device="cuda")
+    B, T, Hq, Hkv, d, W, R = wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, wl.window, wl.R
+    G = Hq // Hkv
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device="cuda")
+    if bank:
+        C = 16
+        rs = synth.normal((B, T, Hq, C), 5, "rs", std=0.25, device="cuda")
+        proj = synth.normal((1, C, R), 5, "proj", std=0.5, device="cuda")
+        o = ops.attn_fwd_bank(x["q"], x["k"], x["v"], rs, proj, W, R, wl.scale, lse=lse)
+        g = ops.attn_bwd_bank(x["q"], x["k"], x["v"], rs, proj, o, lse, x["dout"], W, R, wl.scale)
+    else:
+        o = ops.attn_fwd(x["q"], x["k"], x["v"], x["r"], x["w"], W, R, wl.scale, lse=lse)
+        g = ops.attn_bwd(x["q"], x["k"], x["v"], x["r"], x["w"], o, lse, x["dout"], W, R, wl.scale)
+    torch.cuda.synchronize()
+    b, kv, i0, n = 1, 2, 5000, 64
+    lo, hi = i0 - (W - 1), i0 + n + (W - 1)
+    heads = slice(kv * G, (kv + 1) * G)
+    sl = lambda t: t[b:b + 1, lo:hi].cpu()
+    if bank:
+        r_in, w_in = rs[b:b + 1, lo:hi, heads].cpu(), proj.cpu()
+    else:
+        r_in, w_in = x["r"][b:b + 1, lo:hi, heads].cpu(), x["w"][heads].cpu()
+    ref = O.attn_backward(sl(x["q"])[:, :, heads], sl(x["k"])[:, :, kv:kv + 1], sl(x["v"])[:, :, kv:kv + 1], r_in, w_in,
+                          sl(x["dout"])[:, :, heads], W, R, wl.scale)
+    dr_name = "drs" if bank else "dr"
+    checks = [
+        ("dq", g["dq"][b, i0:i0 + n, heads].double().cpu(), torch.as_tensor(ref["dq"])[0, W - 1:W - 1 + n]),
+        ("dr", g[dr_name][b, i0:i0 + n, heads].double().cpu(), torch.as_tensor(ref["dr"])[0, W - 1:W - 1 + n]),
+        ("dk", g["dk"][b, i0:i0 + n, kv].double().cpu(), torch.as_tensor(ref["dk"])[0, W - 1:W - 1 + n, 0]),
+        ("dv", g["dv"][b, i0:i0 + n, kv].double().cpu(), torch.as_tensor(ref["dv"])[0, W - 1:W - 1 + n, 0]),
+    ]
+    for name, got, want in checks:
+        err = (got - want).abs().max().item()
+        scale = want.abs().max().item()
+        assert err <= 2e-2 * scale + 1e-7, "%s %s: max err %.3e vs max |ref| %.3e" % ("bank" if bank else "rank-1",
+                                                                                     name, err, scale)
