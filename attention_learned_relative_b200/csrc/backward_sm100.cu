@@ -822,6 +822,19 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     float* em = emit + (threadIdx.x >> 5) * kBN;
 #pragma unroll 1
                     for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
+                        // The bank form: this chunk's 32 curve values, loaded ahead of the
+                        // tensor-memory loads so their latencies overlap (values of masked
+                        // cells are not used).
+                        float cw[32];
+                        if constexpr (NCOPY == 0) {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) {
+                                const int c = 32 * ch + k, dist = delta0 + c - t;
+                                cw[k] = (biased && dist >= 0 && dist < p.R && i0 + c < p.T)
+                                            ? __ldg(cstep + c * cstride - (c & 7))
+                                            : 0.0f;
+                            }
+                        }
                         uint32_t sv[32], dv[32];
                         tmem_ld32(st_tm + 32 * ch, sv);
                         tmem_ld32(dpt_tm + 32 * ch, dv);
@@ -839,10 +852,10 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                                 const int dist = delta0 + c - t;
                                 const bool vis = key_ok && dist >= 0 && i0 + c < p.T && (!edge || p.window <= 0 || dist < p.window);
                                 float wv = 0.0f;
-                                if (NCOPY > 0) {
+                                if constexpr (NCOPY > 0) {
                                     if (biased) wv = run[c];
-                                } else if (biased && vis && dist < p.R) {
-                                    wv = __ldg(cstep + c * cstride - (c & 7));
+                                } else {
+                                    wv = cw[e + k];
                                 }
                                 const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
                                 const float pv = vis ? ex2_approx(x) : 0.0f;
