@@ -387,6 +387,18 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 for (int lc = 0; lc < 2; ++lc) {
                     const int ch = 2 * half + lc;   // this half's chunks of 32 columns
                     uint32_t* pk = pk2[lc];
+                    // The bank form: this chunk's curve values (eight aligned groups of four
+                    // distances), loaded ahead of the tensor-memory load.
+                    float4 cv4[8];
+                    if constexpr (NCOPY == 0) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int dlo4 = delta0 + t - (32 * ch + 4 * u) - 3;
+                            cv4[u] = (biased && row_ok && dlo4 + 3 >= 0 && dlo4 < p.R)
+                                         ? __ldg(reinterpret_cast<const float4*>(curve + dlo4))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
                     uint32_t sv[32];
                     tmem_ld32(s_tm + 32 * ch, sv);
                     tmem_ld_wait_regs(sv);
@@ -397,11 +409,9 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                         // group of the padded curve row).
                         const int dlo4 = delta0 + t - (32 * ch + e) - 3;
                         const bool in_curve = row_ok && dlo4 + 3 >= 0 && dlo4 < p.R;
-                        if (NCOPY == 0) {
-                            if (biased && in_curve) {
-                                const float4 v = __ldg(reinterpret_cast<const float4*>(curve + dlo4));
-                                w4[0] = v.w, w4[1] = v.z, w4[2] = v.y, w4[3] = v.x;
-                            }
+                        if constexpr (NCOPY == 0) {
+                            const float4 v = cv4[e / 4];
+                            w4[0] = v.w, w4[1] = v.z, w4[2] = v.y, w4[3] = v.x;
                         } else if (biased) {
                             if constexpr (NCOPY == 4) {
                                 const float4 v = *reinterpret_cast<const float4*>(run + 32 * ch + e);
