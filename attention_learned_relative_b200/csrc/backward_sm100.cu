@@ -1011,49 +1011,67 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const C
 //   dproj[hp, c, d] = sum over the rows of head group hp of rs[row, c] dcv[row, d]
 // (the chain rule through curve = sum_c rs[c] proj[c, :], "Thinking Machines dropped
 // RoPE", recipe step 2).
-constexpr int kDrsRows = 128;    // rows of one (b, h) per block, a thread each
-constexpr int kDrsChunk = 64;    // distances of proj staged per pass
+constexpr int kDrsRows = 128;    // rows of one (b, h) per block
+constexpr int kDrsK = 32;        // distances per pass
 constexpr int kDprojRows = 512;  // rows of one (b, h) per block
 constexpr int kDprojThreads = 256;
 
-__global__ void __launch_bounds__(kDrsRows) bank_drs_kernel(const float* __restrict__ proj, const float* __restrict__ dcv,
-                                                            float* __restrict__ drs, int T, int Hq, int C,
-                                                            int proj_heads, int R, int S) {
-    __shared__ __align__(16) float pj[kDrsChunk][kMaxBankC];   // proj[hp, c, d0 + x] at [x][c]
+// A GEMM tile: 128 rows x 16 functions per block, distances in passes of 32.  Each pass
+// stages the rows' 32 gradient values (a warp reads whole 128-byte row segments) and
+// the functions' 32 values in shared memory; each thread then owns 4 rows x 4
+// functions: per distance, 4 + 1 shared-memory loads feed 16 multiply-adds.
+__global__ void __launch_bounds__(128) bank_drs_kernel(const float* __restrict__ proj, const float* __restrict__ dcv,
+                                                       float* __restrict__ drs, int T, int Hq, int C, int proj_heads,
+                                                       int R, int S) {
+    __shared__ float gs[kDrsK][kDrsRows + 1];                 // [d][row], padded rows
+    __shared__ __align__(16) float ps[kDrsK][kMaxBankC];      // [d][c]
     const int iblocks = (T + kDrsRows - 1) / kDrsRows;
     const int ib = static_cast<int>(blockIdx.x) % iblocks;
     const int bh = static_cast<int>(blockIdx.x) / iblocks;
     const int h = bh % Hq, b = bh / Hq;
-    const int i = ib * kDrsRows + static_cast<int>(threadIdx.x);
-    const bool ok = i < T;
-    const size_t row = (static_cast<size_t>(b) * T + (ok ? i : 0)) * Hq + h;
-    const float* dc = dcv + row * S + (7 - (i & 7));
+    const int i0 = ib * kDrsRows;
+    const int tid = static_cast<int>(threadIdx.x), lane = tid & 31, warp = tid >> 5;
+    const int rg = tid >> 2, cg = tid & 3;          // rows rg + 32u (u < 4), functions 4cg .. 4cg+3
     const float* pr = proj + static_cast<size_t>(proj_heads == 1 ? 0 : h) * C * R;
-    float acc[kMaxBankC];
+    const size_t row_step = static_cast<size_t>(Hq) * S;
+    const float* base = dcv + ((static_cast<size_t>(b) * T + i0) * Hq + h) * S;
+    float acc[4][4];
 #pragma unroll
-    for (int c = 0; c < kMaxBankC; ++c) acc[c] = 0.0f;
-    for (int d0 = 0; d0 < R; d0 += kDrsChunk) {
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.0f;
+    for (int d0 = 0; d0 < R; d0 += kDrsK) {
         __syncthreads();
-        for (int x = threadIdx.x; x < kDrsChunk * kMaxBankC; x += kDrsRows) {
-            const int c = x / kDrsChunk, dd = x % kDrsChunk;
-            pj[dd][c] = (c < C && d0 + dd < R) ? __ldg(pr + static_cast<size_t>(c) * R + d0 + dd) : 0.0f;
+        // Gradient tile: warp w loads rows w, w+4, ..., lane = distance.
+        for (int r = warp; r < kDrsRows; r += 4) {
+            const int i = i0 + r, d = d0 + lane;
+            gs[lane][r] = (i < T && d < R) ? __ldg(base + r * row_step + (7 - (i & 7)) + d) : 0.0f;
+        }
+        for (int x = tid; x < kDrsK * kMaxBankC; x += 128) {
+            const int c = x / kDrsK, dd = x % kDrsK;
+            ps[dd][c] = (c < C && d0 + dd < R) ? __ldg(pr + static_cast<size_t>(c) * R + d0 + dd) : 0.0f;
         }
         __syncthreads();
-        if (!ok) continue;
-        const int dn = min(kDrsChunk, R - d0);
-#pragma unroll 4
-        for (int x = 0; x < dn; ++x) {
-            const float v = __ldg(dc + d0 + x);
+#pragma unroll 8
+        for (int dd = 0; dd < kDrsK; ++dd) {
+            const float4 q = *reinterpret_cast<const float4*>(&ps[dd][4 * cg]);
 #pragma unroll
-            for (int c = 0; c < kMaxBankC; c += 4) {
-                const float4 q = *reinterpret_cast<const float4*>(&pj[x][c]);
-                acc[c] = fmaf(v, q.x, acc[c]), acc[c + 1] = fmaf(v, q.y, acc[c + 1]);
-                acc[c + 2] = fmaf(v, q.z, acc[c + 2]), acc[c + 3] = fmaf(v, q.w, acc[c + 3]);
+            for (int u = 0; u < 4; ++u) {
+                const float g = gs[dd][rg + 32 * u];
+                acc[u][0] = fmaf(g, q.x, acc[u][0]), acc[u][1] = fmaf(g, q.y, acc[u][1]);
+                acc[u][2] = fmaf(g, q.z, acc[u][2]), acc[u][3] = fmaf(g, q.w, acc[u][3]);
             }
         }
     }
-    if (ok)
-        for (int c = 0; c < C; ++c) drs[row * C + c] = acc[c];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = i0 + rg + 32 * u;
+        if (i >= T) continue;
+        float* out = drs + ((static_cast<size_t>(b) * T + i) * Hq + h) * C;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            if (4 * cg + v < C) out[4 * cg + v] = acc[u][v];
+    }
 }
 
 __global__ void __launch_bounds__(kDprojThreads) bank_dproj_kernel(const float* __restrict__ rs,
@@ -1104,7 +1122,7 @@ cudaError_t launch_bank_grads(const float* rs, const float* proj, const float* d
     const long long bh = static_cast<long long>(B) * Hq;
     const long long n1 = bh * ((T + kDrsRows - 1) / kDrsRows), n2 = bh * ((T + kDprojRows - 1) / kDprojRows);
     if (n1 > INT32_MAX || n2 > INT32_MAX) return cudaErrorInvalidValue;
-    bank_drs_kernel<<<static_cast<unsigned>(n1), kDrsRows, 0, stream>>>(proj, dcv, drs, T, Hq, C, proj_heads, R, S);
+    bank_drs_kernel<<<static_cast<unsigned>(n1), 128, 0, stream>>>(proj, dcv, drs, T, Hq, C, proj_heads, R, S);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bank_dproj_kernel<<<static_cast<unsigned>(n2), kDprojThreads, 0, stream>>>(rs, dcv, dproj, T, Hq, C, proj_heads, R,

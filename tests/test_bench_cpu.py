@@ -76,7 +76,7 @@ def test_committed_ncu_summaries_carry_their_source_digest(monkeypatch):
 
 
 def test_default_run_times_every_workload_in_one_line():
-    """The default invocation (the driver's) measures the headline workload and every
+    """The default invocation (no arguments) measures the headline workload and every
     workload in PER_CONFIG; any other --workload times only itself."""
     a = bench.parse_args([])
     assert a.per_config and a.workload == bench.DEFAULT_WORKLOAD
