@@ -33,6 +33,12 @@
 // the copy that makes its run start on an NCOPY-float boundary and reads it with
 // 64- or 128-bit loads.  Copy strides are chosen so that a warp's loads hit
 // distinct banks.
+//
+// Instances: NCOPY in {1, 2, 4} is the rank-1 form with that many table copies;
+// NCOPY = 0 is the shared-bank form, which reads each row's curve (written by
+// bank_rows_kernel, below) from global memory in place of r_i * w.  PAGED reads K
+// and V from a page pool through a block table, with per-sequence chunk offsets and
+// lengths.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
