@@ -10,17 +10,21 @@
 // (the plain derivative of the forward definition: "Thinking Machines dropped RoPE",
 // recipe steps 3-5, for the bias; the pages train the model but print no backward).
 //
-// Two kernels, as in the forward one row of a 128 x 128 tile per thread:
+// Kernels (one row of a 128 x 128 tile per thread, 64 of its columns per warp: two
+// warps share each TMEM lane quadrant):
+//   bwd_dvec_kernel        D_i = dO_i . O_i for every row (and dr zeroed).
 //   bwd_dq_sm100_kernel    per (sequence, query head, 128-row query tile): over the
 //       visible key tiles, S = Q K^T and dP = dO V^T into tensor memory, dl in
 //       registers (dr accumulated with the staged distance table, as the forward adds
-//       the bias), dS = tau scale dl written back over S as bf16, dQ += dS K.  Writes
-//       dq, dr and D_i (for the second kernel).
+//       the bias), dS = tau scale dl written back over S as bf16, dQ += dS K.
 //   bwd_dkv_sm100_kernel   per (sequence, key/value head, 128-key tile): over the
 //       group's query heads and the query tiles that see the keys, S^T = K Q^T and
 //       dP^T = V dO^T, P^T and dS^T in registers (one key row per thread), then
 //       dV += P^T dO and dK += dS^T Q with P^T and dS^T read from tensor memory; dw
-//       summed along the tile's diagonals in shared memory.
+//       summed along the tile's diagonals.
+// The shared-bank form (NCOPY = 0 instances) reads each row's curve in place of
+// r_i * w and writes dL/dcurve instead of dr and dw; bank_drs_kernel and
+// bank_dproj_kernel turn it into the gradients of the coefficients and the bank.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
