@@ -69,9 +69,9 @@ struct BwdTcParams {
     const __nv_bfloat16* o;     // [B, T, Hq, d] forward output
     const __nv_bfloat16* dout;  // [B, T, Hq, d]
     const float* lse;           // [B, Hq, T] forward log-sum-exp
-    float* dvec;                // [B, Hq, T] D_i = dout_i . o_i (written by the dQ kernel)
+    float* dvec;                // [B, Hq, T] D_i = dout_i . o_i (written by bwd_dvec_kernel)
     float* dq;                  // [B, T, Hq, d]
-    float* dr;                  // [B, T, Hq]
+    float* dr;                  // [B, T, Hq] (nullptr in the bank form)
     float* dk;                  // [B, T, Hkv, d]
     float* dv;                  // [B, T, Hkv, d]
     float* dw;                  // [Hq, R], zeroed by the caller, accumulated atomically
