@@ -31,6 +31,8 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
+#include <type_traits>
+
 namespace relbias {
 
 namespace {
@@ -385,71 +387,84 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBM - 1 >= p.window);
                 const int hi = delta0 + t;
                 const int lo = p.window > 0 ? delta0 + t - p.window + 1 : INT_MIN;
+                uint32_t pk2[4][8];   // the chunks' dS: live until the stores are waited for
+                // The chunk loop, compiled with the table bias (a biased tile of the rank-1 form)
+                // and without it, so that no table load sits under a per-chunk branch.  Chunks of
+                // 16 columns keep the bank form's prefetched curve values in registers.
+                auto chunks = [&](auto bias_tag) {
+                    constexpr bool kBiasTab = NCOPY > 0 && decltype(bias_tag)::value;
 #pragma unroll
-                uint32_t pk2[2][16];   // both chunks' dS: live until the stores are waited for
-#pragma unroll
-                for (int lc = 0; lc < 2; ++lc) {
-                    const int ch = 2 * half + lc;   // this half's chunks of 32 columns
-                    uint32_t* pk = pk2[lc];
-                    // The bank form: this chunk's curve values (eight aligned groups of four
-                    // distances), loaded ahead of the tensor-memory load.
-                    float4 cv4[8];
-                    if constexpr (NCOPY == 0) {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int dlo4 = delta0 + t - (32 * ch + 4 * u) - 3;
-                            cv4[u] = (biased && row_ok && dlo4 + 3 >= 0 && dlo4 < p.R)
-                                         ? __ldg(reinterpret_cast<const float4*>(curve + dlo4))
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
-                    }
-                    uint32_t sv[32];
-                    tmem_ld32(s_tm + 32 * ch, sv);
-                    tmem_ld_wait_regs(sv);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        float w4[4] = {0.f, 0.f, 0.f, 0.f};
-                        // Distances of columns c .. c+3 are dlo4+3 .. dlo4 (a 16-byte aligned
-                        // group of the padded curve row).
-                        const int dlo4 = delta0 + t - (32 * ch + e) - 3;
-                        const bool in_curve = row_ok && dlo4 + 3 >= 0 && dlo4 < p.R;
+                    for (int lc = 0; lc < 4; ++lc) {
+                        const int ch = 4 * half + lc;   // this half's chunks of 16 columns
+                        uint32_t* pk = pk2[lc];
+                        // The bank form: this chunk's curve values (four aligned groups of four
+                        // distances), loaded ahead of the tensor-memory load.
+                        float4 cv4[4];
                         if constexpr (NCOPY == 0) {
-                            const float4 v = cv4[e / 4];
-                            w4[0] = v.w, w4[1] = v.z, w4[2] = v.y, w4[3] = v.x;
-                        } else if (biased) {
-                            if constexpr (NCOPY == 4) {
-                                const float4 v = *reinterpret_cast<const float4*>(run + 32 * ch + e);
-                                w4[0] = v.x, w4[1] = v.y, w4[2] = v.z, w4[3] = v.w;
-                            } else if constexpr (NCOPY == 2) {
-                                const float2 a = *reinterpret_cast<const float2*>(run + 32 * ch + e);
-                                const float2 b = *reinterpret_cast<const float2*>(run + 32 * ch + e + 2);
-                                w4[0] = a.x, w4[1] = a.y, w4[2] = b.x, w4[3] = b.y;
-                            } else {
 #pragma unroll
-                                for (int k = 0; k < 4; ++k) w4[k] = run[32 * ch + e + k];
+                            for (int u = 0; u < 4; ++u) {
+                                const int dlo4 = delta0 + t - (16 * ch + 4 * u) - 3;
+                                cv4[u] = (biased && row_ok && dlo4 + 3 >= 0 && dlo4 < p.R)
+                                             ? __ldg(reinterpret_cast<const float4*>(curve + dlo4))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
                             }
                         }
-                        float dl[4];
+                        uint32_t sv[16];
+                        tmem_ld16(s_tm + 16 * ch, sv);
+                        tmem_ld_wait_regs16(sv);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int c = 32 * ch + e + k;
-                            const float x = fmaf(__uint_as_float(sv[e + k]), c1, fmaf(rb, w4[k], -lse2));
-                            const bool vis = !edge || (c <= hi && c >= lo);
-                            const float pr = vis ? ex2_approx(x) : 0.0f;
-                            dl[k] = pr * (__uint_as_float(dp[32 * lc + e + k]) - Di);
-                            if constexpr (NCOPY > 0) dr_acc = fmaf(dl[k], w4[k], dr_acc);
+                        for (int e = 0; e < 16; e += 4) {
+                            float w4[4] = {0.f, 0.f, 0.f, 0.f};
+                            // Distances of columns c .. c+3 are dlo4+3 .. dlo4 (a 16-byte aligned
+                            // group of the padded curve row).
+                            const int dlo4 = delta0 + t - (16 * ch + e) - 3;
+                            const bool in_curve = row_ok && dlo4 + 3 >= 0 && dlo4 < p.R;
+                            if constexpr (NCOPY == 0) {
+                                const float4 v = cv4[e / 4];
+                                w4[0] = v.w, w4[1] = v.z, w4[2] = v.y, w4[3] = v.x;
+                            } else if constexpr (kBiasTab) {
+                                if constexpr (NCOPY == 4) {
+                                    const float4 v = *reinterpret_cast<const float4*>(run + 16 * ch + e);
+                                    w4[0] = v.x, w4[1] = v.y, w4[2] = v.z, w4[3] = v.w;
+                                } else if constexpr (NCOPY == 2) {
+                                    const float2 a = *reinterpret_cast<const float2*>(run + 16 * ch + e);
+                                    const float2 b = *reinterpret_cast<const float2*>(run + 16 * ch + e + 2);
+                                    w4[0] = a.x, w4[1] = a.y, w4[2] = b.x, w4[3] = b.y;
+                                } else {
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k) w4[k] = run[16 * ch + e + k];
+                                }
+                            }
+                            float dl[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int c = 16 * ch + e + k;
+                                const float x = fmaf(__uint_as_float(sv[e + k]), c1, fmaf(rb, w4[k], -lse2));
+                                const bool vis = !edge | ((c <= hi) & (c >= lo));
+                                const float pr = vis ? ex2_approx(x) : 0.0f;
+                                dl[k] = pr * (__uint_as_float(dp[16 * lc + e + k]) - Di);
+                                if constexpr (NCOPY > 0) dr_acc = fmaf(dl[k], w4[k], dr_acc);
+                            }
+                            if (NCOPY == 0 && biased && in_curve)
+                                *reinterpret_cast<float4*>(dcurve + dlo4) =
+                                    make_float4(tau * dl[3], tau * dl[2], tau * dl[1], tau * dl[0]);
+                            pk[e / 2] = pack_bf16x2(dl[0] * ds_scale, dl[1] * ds_scale);
+                            pk[e / 2 + 1] = pack_bf16x2(dl[2] * ds_scale, dl[3] * ds_scale);
                         }
-                        if (NCOPY == 0 && biased && in_curve)
-                            *reinterpret_cast<float4*>(dcurve + dlo4) =
-                                make_float4(tau * dl[3], tau * dl[2], tau * dl[1], tau * dl[0]);
-                        pk[e / 2] = pack_bf16x2(dl[0] * ds_scale, dl[1] * ds_scale);
-                        pk[e / 2 + 1] = pack_bf16x2(dl[2] * ds_scale, dl[3] * ds_scale);
+                        tmem_st8(s_tm + 8 * ch + 32 * half, pk);
                     }
-                    tmem_st16(s_tm + 16 * ch + 32 * half, pk);
+                };
+                if constexpr (NCOPY > 0) {
+                    if (biased)
+                        chunks(std::true_type{});
+                    else
+                        chunks(std::false_type{});
+                } else {
+                    chunks(std::false_type{});
                 }
                 tmem_st_wait();
-                tmem_regs_keep16(pk2[0]);
-                tmem_regs_keep16(pk2[1]);
+#pragma unroll
+                for (int lc = 0; lc < 4; ++lc) tmem_regs_keep8(pk2[lc]);
                 tc_fence_before();
                 // S is double-buffered and dP(g+1) needs only dp_free(g), so a warp can
                 // reach this arrival for tile g while another has yet to arrive for g-1.
@@ -506,8 +521,8 @@ struct BkLayout {
     static constexpr int kV = kK + kTile;
     static constexpr int kQ = kV + kTile;              // 2 stages
     static constexpr int kDO = kQ + 2 * kTile;         // 2 stages
-    static constexpr int kCol = kDO + 2 * kTile;       // per-column constants, 2 buffers of [128] float8
-    static constexpr int kEm = kCol + 2 * kBM * 32;    // per key-row warp: its diagonal sums by column [8][128]
+    static constexpr int kCol = kDO + 2 * kTile;       // per-column constants, 2 buffers of [128] float4
+    static constexpr int kEm = kCol + 2 * kBM * 16;    // per key-row warp: its diagonal sums by column [8][128]
     static constexpr int kDw = kEm + kBkRowWarps * kBN * 4;   // table gradient accumulator [R]
 };
 
@@ -740,7 +755,10 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(t & ~31) << 16;
         const uint32_t st_tm = tmem_base + lane_off, dpt_tm = tmem_base + lane_off + 128,
                        dv_tm = tmem_base + lane_off + 256, dk_tm = tmem_base + lane_off + 384;
-        float4* col = reinterpret_cast<float4*>(smem + L::kCol);   // [2][128] x {c1, rb, lse2, D, dsc, twr, -, -}
+        // Per query column {c1, rb, lse2, D}: one 16-byte load per cell, since these broadcast
+        // loads bound the cell loop.  The cell's other two factors follow from them:
+        // tau * scale = c1 ln 2 and tau * r = rb ln 2 (c1 = tau * scale * log2 e, rb = c1 r / scale).
+        float4* col = reinterpret_cast<float4*>(smem + L::kCol);   // [2][128]
         uint32_t col_phase = 0;
         int ns = 0;
         bool ok = true;
@@ -776,7 +794,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 }
                 for (int qt = qt_lo; qt <= qt_hi; ++qt, ++ns) {
                     const int i0 = qt * kBM;
-                    float4* cb = col + (ns & 1) * 2 * kBM;
+                    float4* cb = col + (ns & 1) * kBM;
                     const float3 cur = nxt;
                     {
                         // The step after this one, and its inputs in flight meanwhile.
@@ -803,11 +821,9 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                         }
                         const float c1 = p.scale_log2 * tau;
                         const float ri = cur.x;
-                        // (the two halves write one float4 each)
                         // (the bank form's curve holds the whole bias: coefficient 1 / scale)
                         const float rcoef = NCOPY > 0 ? ri : 1.0f;
-                        cb[2 * t + half] = half == 0 ? make_float4(c1, rcoef * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z)
-                                                     : make_float4(tau * bp.scale, tau * ri, 0.0f, 0.0f);
+                        if (half == 0) cb[t] = make_float4(c1, rcoef * p.inv_scale * c1, cur.y * 1.4426950408889634f, cur.z);
                     }
                     if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
                     if (!(ok = warp_all(mbar_wait(&bars->sdp_full, ns & 1, abort_flag)))) break;
@@ -817,7 +833,13 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     const int y0 = delta0 - t - kBkDmin;       // table entry of column 0
                     const int cp = y0 & (NCOPY - 1);
                     const float* run = wtab + cp * tstride + (y0 - cp);
-                    const bool edge = delta0 < kBN || (p.window > 0 && delta0 + kBN - 1 >= p.window);
+                    // Query column c sees key row t iff lo <= c <= hi (dist >= 0, inside the
+                    // window, query row inside the sequence, key row inside it).  Integer
+                    // bounds per step, so that a cell's test is two compares and no branch.
+                    int vis_lo = max(0, t - delta0);
+                    int vis_hi = min(kBM - 1, p.T - 1 - i0);
+                    if (p.window > 0) vis_hi = min(vis_hi, t - delta0 + p.window - 1);
+                    if (!key_ok) vis_hi = -1;
                     // The bank form: query row i0 + c's curve at distance delta0 + c - t is
                     // cstep[c * cstride - (c & 7)] (rows (b, i, h) of curve_stride floats, the
                     // row of position i padded by 7 - (i & 7)).
@@ -834,64 +856,78 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     // distinct-address rows of sums to dw instead of one per cell.
                     float zdw = 0.0f;
                     float* em = emit + (threadIdx.x >> 5) * kBN;
+                    // The chunk loop, compiled with the dw conveyor (a biased tile of the rank-1
+                    // form) and without it, so that no warp shuffle sits under a per-cell branch.
+                    // Chunks of 16 columns: with 32, the two tensor-memory loads, the packed
+                    // results and the cells in flight spilled registers.
+                    auto chunks = [&](auto conveyor) {
+                        constexpr bool kConvey = NCOPY > 0 && decltype(conveyor)::value;
 #pragma unroll 1
-                    for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
-                        // The bank form: this chunk's 32 curve values, loaded ahead of the
-                        // tensor-memory loads so their latencies overlap (values of masked
-                        // cells are not used).
-                        float cw[32];
-                        if constexpr (NCOPY == 0) {
+                        for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
+                            // The bank form: this chunk's 16 curve values, loaded ahead of the
+                            // tensor-memory loads so their latencies overlap (values of masked
+                            // cells are not used).
+                            float cw[16];
+                            if constexpr (NCOPY == 0) {
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                const int c = 32 * ch + k, dist = delta0 + c - t;
-                                cw[k] = (biased && dist >= 0 && dist < p.R && i0 + c < p.T)
-                                            ? __ldg(cstep + c * cstride - (c & 7))
-                                            : 0.0f;
-                            }
-                        }
-                        uint32_t sv[32], dv[32];
-                        tmem_ld32(st_tm + 32 * ch, sv);
-                        tmem_ld32(dpt_tm + 32 * ch, dv);
-                        tmem_ld_wait_regs(sv);
-                        tmem_regs_fence(dv);
-                        uint32_t pp[16], pd[16];
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float pr[2], dsv[2];
-#pragma unroll
-                            for (int k = 0; k < 2; ++k) {
-                                const int c = 32 * ch + e + k;
-                                const float4 a = cb[2 * c];
-                                const float4 b2 = cb[2 * c + 1];
-                                const int dist = delta0 + c - t;
-                                const bool vis = key_ok && dist >= 0 && i0 + c < p.T && (!edge || p.window <= 0 || dist < p.window);
-                                float wv = 0.0f;
-                                if constexpr (NCOPY > 0) {
-                                    if (biased) wv = run[c];
-                                } else {
-                                    wv = cw[e + k];
-                                }
-                                const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
-                                const float pv = vis ? ex2_approx(x) : 0.0f;
-                                const float dl = pv * (__uint_as_float(dv[e + k]) - a.w);
-                                pr[k] = pv;
-                                dsv[k] = dl * b2.x;
-                                if (NCOPY > 0 && biased) {
-                                    const float g = (dist >= 0 && dist < p.R) ? dl * b2.y : 0.0f;
-                                    const float up = __shfl_up_sync(0xffffffffu, zdw, 1);
-                                    zdw = g + (lane > 0 ? up : 0.0f);
-                                    if (lane == 31) em[c] = zdw;
+                                for (int k = 0; k < 16; ++k) {
+                                    const int c = 16 * ch + k, dist = delta0 + c - t;
+                                    cw[k] = (biased && dist >= 0 && dist < p.R && i0 + c < p.T)
+                                                ? __ldg(cstep + c * cstride - (c & 7))
+                                                : 0.0f;
                                 }
                             }
-                            pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
-                            pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                            uint32_t sv[16], dv[16];
+                            tmem_ld16(st_tm + 16 * ch, sv);
+                            tmem_ld16(dpt_tm + 16 * ch, dv);
+                            tmem_ld_wait_regs16(sv);
+                            tmem_regs_fence16(dv);
+                            uint32_t pp[8], pd[8];
+#pragma unroll
+                            for (int e = 0; e < 16; e += 2) {
+                                float pr[2], dsv[2];
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) {
+                                    const int c = 16 * ch + e + k;
+                                    const float4 a = cb[c];
+                                    const bool vis = (c >= vis_lo) & (c <= vis_hi);
+                                    float wv = 0.0f;
+                                    if constexpr (NCOPY > 0) {
+                                        if (kConvey) wv = run[c];
+                                    } else {
+                                        wv = cw[e + k];
+                                    }
+                                    const float x = fmaf(__uint_as_float(sv[e + k]), a.x, fmaf(a.y, wv, -a.z));
+                                    const float pv = vis ? ex2_approx(x) : 0.0f;
+                                    const float dl = pv * (__uint_as_float(dv[e + k]) - a.w);
+                                    pr[k] = pv;
+                                    dsv[k] = dl * (a.x * kLn2);
+                                    if constexpr (kConvey) {
+                                        // Every cell of a diagonal has one distance: the range
+                                        // [0, R) is checked once, where the diagonal's sum is added.
+                                        const float up = __shfl_up_sync(0xffffffffu, zdw, 1);
+                                        zdw = fmaf(dl, a.y, lane > 0 ? up : 0.0f);   // x ln 2 at the flush
+                                        if (lane == 31) em[c] = zdw;
+                                    }
+                                }
+                                pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
+                                pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                            }
+                            tmem_st8(st_tm + 8 * ch + 32 * half, pp);
+                            tmem_st8(dpt_tm + 8 * ch + 32 * half, pd);
+                            // pp and pd are this loop iteration's registers: wait before reuse.
+                            tmem_st_wait();
+                            tmem_regs_keep8(pp);
+                            tmem_regs_keep8(pd);
                         }
-                        tmem_st16(st_tm + 16 * ch + 32 * half, pp);
-                        tmem_st16(dpt_tm + 16 * ch + 32 * half, pd);
-                        // pp and pd are this loop iteration's registers: wait before reuse.
-                        tmem_st_wait();
-                        tmem_regs_keep16(pp);
-                        tmem_regs_keep16(pd);
+                    };
+                    if constexpr (NCOPY > 0) {
+                        if (biased)
+                            chunks(std::true_type{});
+                        else
+                            chunks(std::false_type{});
+                    } else {
+                        chunks(std::false_type{});
                     }
                     tmem_st_wait();
                     tc_fence_before();
@@ -912,10 +948,11 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     }
                 }
                 if (!ok) break;
-                // This head's table gradient from this key tile, into the output.
+                // This head's table gradient from this key tile, into the output (dw_s holds
+                // sums of dl rb; tau r = rb ln 2).
                 if (!(ok = tab_meet(&bars->col_sync, col_phase, abort_flag))) break;
                 for (int x = threadIdx.x; NCOPY > 0 && x < p.R; x += kBkRowWarps * 32)
-                    if (dw_s[x] != 0.0f) atomicAdd(bp.dw + static_cast<size_t>(h) * p.R + x, dw_s[x]);
+                    if (dw_s[x] != 0.0f) atomicAdd(bp.dw + static_cast<size_t>(h) * p.R + x, dw_s[x] * kLn2);
             }
             if (!ok) break;
             // Epilogue: the key row's dk and dv (fp32).
