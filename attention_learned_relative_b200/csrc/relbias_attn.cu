@@ -774,7 +774,7 @@ extern "C" int relbias_set_wait_limit_ns(unsigned long long ns) {
     return e == cudaSuccess ? RELBIAS_OK : cuda_fail(e, "setting the wait limit");
 }
 
-extern "C" int relbias_version(void) { return 710; }
+extern "C" int relbias_version(void) { return 701; }
 
 // The allocation-free decode variant (its own file: it owns a static device array).
 #include "decode_noalloc.cu"
