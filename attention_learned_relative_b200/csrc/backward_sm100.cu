@@ -883,6 +883,11 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                             tmem_ld_wait_regs16(sv);
                             tmem_regs_fence16(dv);
                             uint32_t pp[8], pd[8];
+                            // Lane 31's finished diagonal sums by column, kept in registers and
+                            // stored when the chunk ends: a store per column sat between the
+                            // next column's shared-memory loads and this column's sum, which
+                            // chained the columns' latencies.
+                            float emr[16];
 #pragma unroll
                             for (int e = 0; e < 16; e += 2) {
                                 float pr[2], dsv[2];
@@ -907,11 +912,17 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                                         // [0, R) is checked once, where the diagonal's sum is added.
                                         const float up = __shfl_up_sync(0xffffffffu, zdw, 1);
                                         zdw = fmaf(dl, a.y, lane > 0 ? up : 0.0f);   // x ln 2 at the flush
-                                        if (lane == 31) em[c] = zdw;
+                                        emr[e + k] = zdw;
                                     }
                                 }
                                 pp[e / 2] = pack_bf16x2(pr[0], pr[1]);
                                 pd[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                            }
+                            if (kConvey && lane == 31) {
+                                float4* e4 = reinterpret_cast<float4*>(em + 16 * ch);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    e4[q] = make_float4(emr[4 * q], emr[4 * q + 1], emr[4 * q + 2], emr[4 * q + 3]);
                             }
                             tmem_st8(st_tm + 8 * ch + 32 * half, pp);
                             tmem_st8(dpt_tm + 8 * ch + 32 * half, pd);
