@@ -91,25 +91,31 @@ struct TileCursor {
     __device__ __forceinline__ int j0() const { return j_first + t * kBN; }
 };
 
-// D_i = dO_i . O_i for every row (b, i, h), into dvec [B, Hq, T], and dr zeroed: one
-// warp per row.
+// D_i = dO_i . O_i for every row (b, i, h), into dvec [B, Hq, T], and dr zeroed.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout, float* __restrict__ dvec,
                                                        float* __restrict__ dr, int B, int T, int Hq) {
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // (b * T + i) * Hq + h
-    const int lane = threadIdx.x & 31;
-    if (row >= static_cast<long long>(B) * T * Hq) return;
+    // D / 8 lanes per row, 16 bytes of o and of dout each (rows are 16-byte aligned).
+    constexpr int kLanes = D / 8;
+    const long long row = static_cast<long long>(blockIdx.x) * (256 / kLanes) + threadIdx.x / kLanes;   // (b * T + i) * Hq + h
+    const int sub = threadIdx.x % kLanes;
+    const bool ok = row < static_cast<long long>(B) * T * Hq;
     float acc = 0.0f;
+    if (ok) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + sub);
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + sub);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int u = lane * 2; u < D; u += 64) {
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + row * D + u));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + row * D + u));
-        acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+        for (int u = 0; u < 4; ++u) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[u]));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[u]));
+            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (ok && sub == 0) {
         const int h = static_cast<int>(row % Hq);
         const long long bi = row / Hq;
         const int i = static_cast<int>(bi % T), b = static_cast<int>(bi / T);
@@ -1037,8 +1043,9 @@ cudaError_t launch_bwd_tc(const CUtensorMap& tq, const CUtensorMap& tdo, const C
                           const CUtensorMap& tv, const PrefillParams& p_dq, const PrefillParams& p_dkv,
                           const BwdTcParams& bp, int grid, cudaStream_t stream) {
     const long long rows = static_cast<long long>(p_dq.B) * p_dq.T * p_dq.Hq;
-    bwd_dvec_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(bp.o, bp.dout, bp.dvec, bp.dr,
-                                                                                 p_dq.B, p_dq.T, p_dq.Hq);
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    bwd_dvec_kernel<D><<<static_cast<unsigned>((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(
+        bp.o, bp.dout, bp.dvec, bp.dr, p_dq.B, p_dq.T, p_dq.Hq);
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
     const int g_dq = std::min(grid, p_dq.total_items), g_dkv = std::min(grid, p_dkv.total_items);
