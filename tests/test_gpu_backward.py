@@ -63,6 +63,9 @@ CASES = [
     (torch.bfloat16, 2, 200, 4, 4, 128, 0, 300, 100),   # group 1, R beyond T, temperature
     (torch.bfloat16, 1, 129, 4, 2, 128, 64, 32, 0),     # one tile plus one row, window < tile
     (torch.bfloat16, 1, 1024, 32, 4, 128, 512, 512, 0), # the local layer's 32 / 4 head layout
+    (torch.bfloat16, 1, 700, 8, 2, 128, 512, 512, 300),  # window and temperature together
+    (torch.bfloat16, 1, 2300, 4, 2, 128, 0, 2048, 0),    # the largest R, global layer, ragged tail
+    (torch.bfloat16, 1, 600, 4, 2, 64, 200, 64, 0),      # d = 64, window not a tile multiple, R < window
 ]
 
 
@@ -118,6 +121,8 @@ BANK_CASES = [
     (1, 640, 8, 2, 128, 512, 512, 16, 8, 0),     # a bank per head, the local layer's window
     (2, 200, 6, 3, 64, 0, 150, 5, 1, 100),       # d = 64, odd group, R not a multiple of 8, temperature
     (1, 129, 4, 2, 128, 64, 30, 3, 4, 0),        # one tile plus one row, window < tile
+    (1, 700, 4, 2, 128, 512, 512, 16, 1, 300),   # window and temperature together
+    (1, 1300, 4, 2, 128, 0, 1024, 16, 1, 0),     # the global layer's R, ragged tail
 ]
 
 
