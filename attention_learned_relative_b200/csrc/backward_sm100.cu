@@ -496,9 +496,7 @@ __global__ void __launch_bounds__(kBqThreads, 1)
                 if (row_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dqrow + c + e) =
-                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                                        __uint_as_float(v[e + 3]));
+                        st_global_v4(dqrow + c + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
                 }
             }
             tc_fence_before();
@@ -986,12 +984,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (key_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
-                        *reinterpret_cast<float4*>(bp.dk + krow * D + c + e) = make_float4(
-                            __uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
-                            __uint_as_float(a[e + 3]));
-                        *reinterpret_cast<float4*>(bp.dv + krow * D + c + e) = make_float4(
-                            __uint_as_float(b[e]), __uint_as_float(b[e + 1]), __uint_as_float(b[e + 2]),
-                            __uint_as_float(b[e + 3]));
+                        st_global_v4(bp.dk + krow * D + c + e, a[e], a[e + 1], a[e + 2], a[e + 3]);
+                        st_global_v4(bp.dv + krow * D + c + e, b[e], b[e + 1], b[e + 2], b[e + 3]);
                     }
                 }
             }

@@ -837,10 +837,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         st_global_v8(orow + c, packed);
                         st_global_v8(orow + c + 16, packed + 8);
                     } else {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                            st_global_v4(orow + c + 8 * e, packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
+                                         packed[4 * e + 3]);
                     }
                 }
             }
